@@ -1,0 +1,214 @@
+/*
+ * dsa_indexer.h - C ABI of the B200 (sm_100a) DeepSeek Sparse Attention lightning indexer,
+ * its top-k selection, IndexCache cross-layer index reuse and the cross-layer top-k overlap.
+ *
+ * What is computed (pages by title and section):
+ *   "IndexShare deep-dive report" (深度解读报告) §1.1: the lightning indexer is a multi-head,
+ *   ReLU-gated dot product over FP8 inputs that scores the whole prefix and keeps the top-k
+ *   keys (k = 2048 in the abstract). It is read here as
+ *       I[t,s] = sum_j w[t,j] * ReLU(q[t,j] . k[s]),
+ *       q[t,j] = q_scale[t] * e4m3(q8[t][j][:]),   k[s] = k_scale[s] * e4m3(k8[s][:]),
+ *   over the causal prefix s <= t ("ADIndex以分组蒸馏重构长上下文稀疏注意力索引", section
+ *   索引器为何成为长上下文瓶颈). Each query keeps the top-k keys, ties going to the lower key
+ *   index; rows are written by (score descending, index ascending), and a row with fewer
+ *   than topk visible keys is padded with index -1 (score -inf).
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers (or managed memory) of the current CUDA
+ *     device, row-major and densely packed as stated. The caller owns every buffer,
+ *     including the workspace; the library allocates no device memory and keeps no state
+ *     between calls. Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and runs asynchronously; outputs are valid once the stream reaches them.
+ *   - FP8 inputs are OCP E4M3 byte codes; the NaN codes 0x7F / 0xFF are not valid input.
+ *     Scales must be finite and > 0.
+ *   - Arguments are validated on the host before anything is enqueued; a rejected call
+ *     returns DSA_ERR_INVALID (malformed) or DSA_ERR_UNSUPPORTED (valid but not built)
+ *     and enqueues nothing. A failed CUDA runtime call returns DSA_ERR_CUDA.
+ *   - Device-side checks (block-table entries, sequence lengths, index ranges) and
+ *     bounded pipeline waits record the FIRST failure in the workspace header; read it
+ *     with dsa_read_device_status. Kernels never trap and never wait without a bound
+ *     (env DSA_WAIT_BUDGET_NS, default 2e9 ns per wait).
+ *   - A workspace's first DSA_WS_HEADER_BYTES must be zeroed once before first use
+ *     (dsa_workspace_init). Calls that share a workspace must not overlap on the GPU.
+ *   - Supported shapes: (H, d) in {(8, 64), (64, 128)}, 1 <= topk <= 2048.
+ */
+#ifndef DSA_INDEXER_H
+#define DSA_INDEXER_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DSA_API __attribute__((visibility("default")))
+
+#define DSA_ABI_VERSION 1
+#define DSA_WS_HEADER_BYTES 256
+#define DSA_MAX_TOPK 2048
+#define DSA_MAX_LAYERS 64
+
+typedef enum dsa_status {
+  DSA_OK = 0,
+  DSA_ERR_INVALID = 1,     /* malformed argument (null, size, alignment, pattern) */
+  DSA_ERR_UNSUPPORTED = 2, /* well-formed but not supported by this build (H, d, topk) */
+  DSA_ERR_CUDA = 3,        /* a CUDA runtime / driver call failed */
+  DSA_ERR_TIMEOUT = 4,     /* device-side: a pipeline wait exceeded its bound */
+  DSA_ERR_DEVICE = 5       /* device-side: an input check failed (see detail) */
+} dsa_status;
+
+enum { DSA_MODE_PREFILL = 0, DSA_MODE_DECODE = 1 };
+
+/* Library ABI version (DSA_ABI_VERSION). */
+DSA_API int32_t dsa_abi_version(void);
+
+/* Static description of a status code; never NULL. */
+DSA_API const char* dsa_status_string(int32_t status);
+
+/* Zeroes the workspace header (the first DSA_WS_HEADER_BYTES) on `stream`.
+ * workspace_bytes must be >= DSA_WS_HEADER_BYTES. */
+DSA_API dsa_status dsa_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then returns in *status_out / *detail_out the first device-side
+ * failure recorded in the workspace header since it was last cleared (DSA_OK / 0 if
+ * none) and clears it. Either output pointer may be NULL. */
+DSA_API dsa_status dsa_read_device_status(void* workspace, void* stream, int32_t* status_out,
+                                          int32_t* detail_out);
+
+/* ---------------------------------------------------------------------------------------
+ * Prefill indexer ("IndexShare deep-dive report" §1.1; "Index Share逻辑详解" §2: every
+ * layer scores the whole length and takes the top-k).
+ *
+ * Queries i = 0..Lq-1 sit at positions t = q_pos0 + i and see keys s = 0..t (a chunk of a
+ * longer prefill is one call with q_pos0 > 0 against all keys before its end; the result
+ * equals the unchunked one).
+ *   q        [Lq][H][d]   u8 E4M3, 16-byte aligned      q_scale [Lq]  f32
+ *   w        [Lq][H]      f32 head weights
+ *   k        [Lk][d]      u8 E4M3, 16-byte aligned      k_scale [Lk]  f32
+ *   out_idx  [Lq][topk]   i32, written                   out_score [Lq][topk] f32 or NULL
+ * Requires q_pos0 >= 0, Lq >= 1, q_pos0 + Lq <= Lk.
+ * workspace: >= dsa_prefill_workspace_bytes(Lq, H, d, topk) bytes, 256-byte aligned.
+ * -------------------------------------------------------------------------------------*/
+DSA_API size_t dsa_prefill_workspace_bytes(int32_t Lq, int32_t H, int32_t d, int32_t topk);
+
+DSA_API dsa_status dsa_indexer_prefill(const uint8_t* q, const float* q_scale, const float* w,
+                                       const uint8_t* k, const float* k_scale, int32_t Lk,
+                                       int32_t q_pos0, int32_t Lq, int32_t H, int32_t d,
+                                       int32_t topk, int32_t* out_idx, float* out_score,
+                                       void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Decode indexer ("Index Share逻辑详解" §2: the decode step runs the indexer in every layer
+ * at every step; "多层索引器" abstract: the indexer scans the whole cache and keeps
+ * k = 2048 tokens).
+ *
+ * Request b has one new query at position seq_lens[b]-1 whose own key is already cached;
+ * it scores all seq_lens[b] cached keys. Logical key s of request b lives in physical
+ * block block_table[b][s / block_size], slot s % block_size.
+ *   q             [B][H][d]                      u8 E4M3      q_scale [B] f32, w [B][H] f32
+ *   k_cache       [n_blocks][block_size][d]      u8 E4M3, 16-byte aligned
+ *   k_scale_cache [n_blocks][block_size]         f32
+ *   block_table   [B][max_blocks]                i32 (entries past a request's last block
+ *                                                 are not read)
+ *   seq_lens      [B]                            i32, 1 <= seq_lens[b] <= max_blocks*block_size
+ *   out_idx       [B][topk] i32 logical positions;  out_score [B][topk] f32 or NULL
+ * block_size must be 64. A block-table entry outside [0, n_blocks) or a bad length is
+ * recorded as DSA_ERR_DEVICE (the request's keys are then read from block 0 / clamped).
+ * workspace: >= dsa_decode_workspace_bytes(B, max_blocks*block_size, H, d, topk) bytes.
+ * -------------------------------------------------------------------------------------*/
+DSA_API size_t dsa_decode_workspace_bytes(int32_t B, int32_t max_len, int32_t H, int32_t d,
+                                          int32_t topk);
+
+DSA_API dsa_status dsa_indexer_decode(const uint8_t* q, const float* q_scale, const float* w,
+                                      const uint8_t* k_cache, const float* k_scale_cache,
+                                      int32_t n_blocks, int32_t block_size,
+                                      const int32_t* block_table, int32_t max_blocks,
+                                      const int32_t* seq_lens, int32_t B, int32_t H, int32_t d,
+                                      int32_t topk, int32_t* out_idx, float* out_score,
+                                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * IndexCache layer driver ("IndexShare deep-dive report" §2.1: Full layers run the indexer
+ * and overwrite the cached indices, Shared layers take T <- T_f(l) with
+ * f(l) = max{j < l : c_j = F}, the first layer is always F, and the cache costs no extra
+ * memory; "Index Share逻辑详解" §4.2: one branch per layer).
+ *
+ * pattern: n_layers characters over {F, S}, first 'F' (no whitespace).
+ * shape:   the per-layer call shape. mode = DSA_MODE_PREFILL uses H, d, topk, Lk, q_pos0,
+ *          Lq; mode = DSA_MODE_DECODE uses H, d, topk, n_blocks, block_size, block_table,
+ *          max_blocks, seq_lens, B.
+ * layers:  [n_layers] per-layer inputs; entries of S layers are not read. For decode,
+ *          k / k_scale are that layer's paged k_cache / k_scale_cache.
+ * f_bufs:  output index buffers, each [rows][topk] i32 (rows = Lq or B). n_fbufs = 1: every
+ *          F layer overwrites f_bufs[0] (the pages' single cache). n_fbufs = number of F
+ *          layers: the m-th F layer writes f_bufs[m] and all layer outputs stay readable.
+ * out_layer_idx: [n_layers] host array, filled with the buffer holding each layer's indices
+ *          (an S layer gets its source F layer's buffer: no copy, no launch).
+ * after_layer: optional host callback invoked after layer l's work has been ENQUEUED (not
+ *          completed) with the buffer holding layer l's indices; work the callback enqueues
+ *          on the same stream runs before the next F layer overwrites a shared buffer.
+ * workspace: >= dsa_indexcache_workspace_bytes(shape) bytes (one layer's worth, reused).
+ * -------------------------------------------------------------------------------------*/
+typedef struct dsa_layer_inputs {
+  const uint8_t* q;
+  const float* q_scale;
+  const float* w;
+  const uint8_t* k;       /* prefill keys [Lk][d] or decode k_cache [n_blocks][block_size][d] */
+  const float* k_scale;   /* prefill [Lk] or decode k_scale_cache [n_blocks][block_size]     */
+  float* out_score;       /* optional [rows][topk] scores of this layer, or NULL             */
+} dsa_layer_inputs;
+
+typedef struct dsa_indexer_shape {
+  int32_t mode;
+  int32_t H, d, topk;
+  int32_t Lk, q_pos0, Lq;                 /* prefill */
+  int32_t n_blocks, block_size;           /* decode  */
+  const int32_t* block_table;
+  int32_t max_blocks;
+  const int32_t* seq_lens;
+  int32_t B;
+} dsa_indexer_shape;
+
+typedef void (*dsa_after_layer_fn)(int32_t layer, const int32_t* layer_idx, void* user);
+
+DSA_API size_t dsa_indexcache_workspace_bytes(const dsa_indexer_shape* shape);
+
+DSA_API dsa_status indexcache_run(const char* pattern, int32_t n_layers,
+                                  const dsa_indexer_shape* shape, const dsa_layer_inputs* layers,
+                                  int32_t* const* f_bufs, int32_t n_fbufs,
+                                  const int32_t** out_layer_idx, dsa_after_layer_fn after_layer,
+                                  void* user, void* workspace, size_t workspace_bytes,
+                                  void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Cross-layer top-k overlap ("IndexShare deep-dive report" §1.2: the overlap of layers i
+ * and j is |T(i) ∩ T(j)| / k; adjacent layers overlap 70-100% in blocks).
+ *
+ * layer_idx: HOST array of n_layers (<= DSA_MAX_LAYERS) device pointers, each [rows][topk]
+ *          i32 index rows as the indexer writes them (distinct entries in [0, n_keys), -1
+ *          padding). Pointers may repeat (aliased S layers).
+ * out_counts [n_layers][n_layers] u64: C[i][j] = sum over rows of |T_i(row) ∩ T_j(row)|.
+ * out_valid  [1] u64: V = number of non-negative entries of layer 0.
+ * out_overlap [n_layers][n_layers] f64 = C / V, or NULL.
+ * An entry outside [-1, n_keys) is skipped and recorded as DSA_ERR_DEVICE.
+ * workspace: >= DSA_WS_HEADER_BYTES bytes. n_keys <= 1,600,000.
+ * -------------------------------------------------------------------------------------*/
+DSA_API dsa_status topk_overlap(const int32_t* const* layer_idx, int32_t n_layers, int32_t rows,
+                                int32_t topk, int32_t n_keys, uint64_t* out_counts,
+                                uint64_t* out_valid, double* out_overlap, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Failure-detection self-test (no counterpart on the pages): launches one CTA that waits,
+ * with the given bound, on an mbarrier that nothing completes, so that the bounded-wait
+ * path records DSA_ERR_TIMEOUT in the workspace header and the kernel returns normally.
+ * -------------------------------------------------------------------------------------*/
+DSA_API dsa_status dsa_selftest_wait_timeout(void* workspace, size_t workspace_bytes,
+                                             uint64_t budget_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_INDEXER_H */

@@ -1,0 +1,273 @@
+// C-ABI entry points: host-side validation, workspace sizing, tensor-map encoding, the
+// IndexCache layer driver and device-status reporting. No device memory is allocated here.
+#include <cstdlib>
+#include <cstring>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace dsa {
+
+namespace {
+
+uint64_t wait_budget_ns() {
+  const char* env = std::getenv("DSA_WAIT_BUDGET_NS");
+  if (env && *env) {
+    char* end = nullptr;
+    unsigned long long v = std::strtoull(env, &end, 10);
+    if (end && *end == '\0' && v > 0) return static_cast<uint64_t>(v);
+  }
+  return 2000000000ull;
+}
+
+int current_num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  return n;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool prefill_shape_supported(int H, int d) { return (H == 64 && d == 128) || (H == 8 && d == 64); }
+
+dsa_status check_prefill(const uint8_t* q, const float* q_scale, const float* w, const uint8_t* k,
+                         const float* k_scale, int32_t Lk, int32_t q_pos0, int32_t Lq, int32_t H,
+                         int32_t d, int32_t topk, const int32_t* out_idx) {
+  if (!q || !q_scale || !w || !k || !k_scale || !out_idx) return DSA_ERR_INVALID;
+  if (Lq < 1 || Lk < 1 || q_pos0 < 0 || static_cast<int64_t>(q_pos0) + Lq > Lk) return DSA_ERR_INVALID;
+  if (topk < 1 || H < 1 || d < 1) return DSA_ERR_INVALID;
+  if (!aligned(q, 16) || !aligned(k, 16)) return DSA_ERR_INVALID;
+  if (!prefill_shape_supported(H, d) || topk > DSA_MAX_TOPK) return DSA_ERR_UNSUPPORTED;
+  return DSA_OK;
+}
+
+dsa_status check_decode(const uint8_t* q, const float* q_scale, const float* w,
+                        const uint8_t* k_cache, const float* k_scale_cache, int32_t n_blocks,
+                        int32_t block_size, const int32_t* block_table, int32_t max_blocks,
+                        const int32_t* seq_lens, int32_t B, int32_t H, int32_t d, int32_t topk,
+                        const int32_t* out_idx) {
+  if (!q || !q_scale || !w || !k_cache || !k_scale_cache || !block_table || !seq_lens || !out_idx)
+    return DSA_ERR_INVALID;
+  if (B < 1 || n_blocks < 1 || max_blocks < 1 || block_size < 1 || topk < 1 || H < 1 || d < 1)
+    return DSA_ERR_INVALID;
+  if (static_cast<int64_t>(max_blocks) * block_size > INT32_MAX) return DSA_ERR_INVALID;
+  if (!aligned(q, 16) || !aligned(k_cache, 16)) return DSA_ERR_INVALID;
+  if (!(H == 64 && d == 128) || block_size != 64 || topk > DSA_MAX_TOPK) return DSA_ERR_UNSUPPORTED;
+  return DSA_OK;
+}
+
+}  // namespace
+
+bool encode_tmap_2d_u8(CUtensorMap* map, const void* base, uint64_t row_bytes, uint64_t rows,
+                       uint32_t box_rows) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  if (!encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult qres;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qres) != cudaSuccess ||
+        qres != cudaDriverEntryPointSuccess || !fn)
+      return false;
+    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  const cuuint64_t dims[2] = {row_bytes, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(row_bytes), box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle swz =
+      row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  return encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace dsa
+
+using namespace dsa;
+
+extern "C" {
+
+DSA_API int32_t dsa_abi_version(void) { return DSA_ABI_VERSION; }
+
+DSA_API const char* dsa_status_string(int32_t status) {
+  switch (status) {
+    case DSA_OK: return "ok";
+    case DSA_ERR_INVALID: return "invalid argument";
+    case DSA_ERR_UNSUPPORTED: return "unsupported shape";
+    case DSA_ERR_CUDA: return "CUDA error";
+    case DSA_ERR_TIMEOUT: return "device wait timed out";
+    case DSA_ERR_DEVICE: return "device-side input check failed";
+    default: return "unknown status";
+  }
+}
+
+DSA_API dsa_status dsa_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
+  if (!workspace || workspace_bytes < DSA_WS_HEADER_BYTES) return DSA_ERR_INVALID;
+  return cuda_status(
+      cudaMemsetAsync(workspace, 0, DSA_WS_HEADER_BYTES, static_cast<cudaStream_t>(stream)));
+}
+
+DSA_API dsa_status dsa_read_device_status(void* workspace, void* stream, int32_t* status_out,
+                                          int32_t* detail_out) {
+  if (!workspace) return DSA_ERR_INVALID;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t h[2] = {0, 0};
+  if (cudaStreamSynchronize(s) != cudaSuccess) return DSA_ERR_CUDA;
+  if (cudaMemcpyAsync(h, workspace, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess) return DSA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return DSA_ERR_CUDA;
+  if (cudaMemsetAsync(workspace, 0, sizeof(h), s) != cudaSuccess) return DSA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return DSA_ERR_CUDA;
+  if (status_out) *status_out = static_cast<int32_t>(h[0]);
+  if (detail_out) *detail_out = static_cast<int32_t>(h[1]);
+  return DSA_OK;
+}
+
+DSA_API size_t dsa_prefill_workspace_bytes(int32_t Lq, int32_t H, int32_t d, int32_t topk) {
+  if (Lq < 1 || topk < 1 || topk > DSA_MAX_TOPK || !prefill_shape_supported(H, d)) return 0;
+  const int sms = current_num_sms();
+  if (sms < 1) return 0;
+  return prefill_workspace_bytes(Lq, H, d, topk, sms);
+}
+
+DSA_API dsa_status dsa_indexer_prefill(const uint8_t* q, const float* q_scale, const float* w,
+                                       const uint8_t* k, const float* k_scale, int32_t Lk,
+                                       int32_t q_pos0, int32_t Lq, int32_t H, int32_t d,
+                                       int32_t topk, int32_t* out_idx, float* out_score,
+                                       void* workspace, size_t workspace_bytes, void* stream) {
+  dsa_status st = check_prefill(q, q_scale, w, k, k_scale, Lk, q_pos0, Lq, H, d, topk, out_idx);
+  if (st != DSA_OK) return st;
+  if (!workspace || !aligned(workspace, 256)) return DSA_ERR_INVALID;
+  const int sms = current_num_sms();
+  if (sms < 1) return DSA_ERR_CUDA;
+  if (workspace_bytes < prefill_workspace_bytes(Lq, H, d, topk, sms)) return DSA_ERR_INVALID;
+  PrefillLaunch a{q, q_scale, w, k, k_scale, Lk, q_pos0, Lq, H, d, topk, out_idx, out_score,
+                  workspace, workspace_bytes, static_cast<cudaStream_t>(stream), wait_budget_ns(), sms};
+  return launch_prefill(a);
+}
+
+DSA_API size_t dsa_decode_workspace_bytes(int32_t B, int32_t max_len, int32_t H, int32_t d,
+                                          int32_t topk) {
+  if (B < 1 || max_len < 1 || topk < 1) return 0;
+  return decode_workspace_bytes(B, max_len, H, d, topk);
+}
+
+DSA_API dsa_status dsa_indexer_decode(const uint8_t* q, const float* q_scale, const float* w,
+                                      const uint8_t* k_cache, const float* k_scale_cache,
+                                      int32_t n_blocks, int32_t block_size,
+                                      const int32_t* block_table, int32_t max_blocks,
+                                      const int32_t* seq_lens, int32_t B, int32_t H, int32_t d,
+                                      int32_t topk, int32_t* out_idx, float* out_score,
+                                      void* workspace, size_t workspace_bytes, void* stream) {
+  dsa_status st = check_decode(q, q_scale, w, k_cache, k_scale_cache, n_blocks, block_size,
+                               block_table, max_blocks, seq_lens, B, H, d, topk, out_idx);
+  if (st != DSA_OK) return st;
+  if (!workspace || !aligned(workspace, 256)) return DSA_ERR_INVALID;
+  if (workspace_bytes < decode_workspace_bytes(B, max_blocks * block_size, H, d, topk)) return DSA_ERR_INVALID;
+  const int sms = current_num_sms();
+  if (sms < 1) return DSA_ERR_CUDA;
+  DecodeLaunch a{q, q_scale, w, k_cache, k_scale_cache, n_blocks, block_size, block_table,
+                 max_blocks, seq_lens, B, H, d, topk, out_idx, out_score, workspace,
+                 workspace_bytes, static_cast<cudaStream_t>(stream), wait_budget_ns(), sms};
+  return launch_decode(a);
+}
+
+DSA_API size_t dsa_indexcache_workspace_bytes(const dsa_indexer_shape* shape) {
+  if (!shape) return 0;
+  if (shape->mode == DSA_MODE_PREFILL)
+    return dsa_prefill_workspace_bytes(shape->Lq, shape->H, shape->d, shape->topk);
+  if (shape->mode == DSA_MODE_DECODE) {
+    if (static_cast<int64_t>(shape->max_blocks) * shape->block_size > INT32_MAX) return 0;
+    return dsa_decode_workspace_bytes(shape->B, shape->max_blocks * shape->block_size, shape->H,
+                                      shape->d, shape->topk);
+  }
+  return 0;
+}
+
+DSA_API dsa_status indexcache_run(const char* pattern, int32_t n_layers,
+                                  const dsa_indexer_shape* shape, const dsa_layer_inputs* layers,
+                                  int32_t* const* f_bufs, int32_t n_fbufs,
+                                  const int32_t** out_layer_idx, dsa_after_layer_fn after_layer,
+                                  void* user, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  if (!pattern || !shape || !layers || !f_bufs || !out_layer_idx || n_layers < 1) return DSA_ERR_INVALID;
+  if (static_cast<int64_t>(std::strlen(pattern)) != n_layers) return DSA_ERR_INVALID;
+  int n_full = 0;
+  for (int l = 0; l < n_layers; ++l) {
+    if (pattern[l] == 'F') ++n_full;
+    else if (pattern[l] != 'S') return DSA_ERR_INVALID;
+  }
+  if (pattern[0] != 'F') return DSA_ERR_INVALID;  // the first layer is always Full
+  if (n_fbufs != 1 && n_fbufs != n_full) return DSA_ERR_INVALID;
+  for (int m = 0; m < n_fbufs; ++m)
+    if (!f_bufs[m]) return DSA_ERR_INVALID;
+  if (shape->mode != DSA_MODE_PREFILL && shape->mode != DSA_MODE_DECODE) return DSA_ERR_INVALID;
+  // Validate every Full layer before anything is enqueued.
+  for (int l = 0; l < n_layers; ++l) {
+    if (pattern[l] != 'F') continue;
+    const dsa_layer_inputs& in = layers[l];
+    dsa_status st;
+    if (shape->mode == DSA_MODE_PREFILL)
+      st = check_prefill(in.q, in.q_scale, in.w, in.k, in.k_scale, shape->Lk, shape->q_pos0,
+                         shape->Lq, shape->H, shape->d, shape->topk, f_bufs[0]);
+    else
+      st = check_decode(in.q, in.q_scale, in.w, in.k, in.k_scale, shape->n_blocks,
+                        shape->block_size, shape->block_table, shape->max_blocks, shape->seq_lens,
+                        shape->B, shape->H, shape->d, shape->topk, f_bufs[0]);
+    if (st != DSA_OK) return st;
+  }
+  const size_t need = dsa_indexcache_workspace_bytes(shape);
+  if (!workspace || need == 0 || workspace_bytes < need || !aligned(workspace, 256)) return DSA_ERR_INVALID;
+
+  int m = 0;
+  const int32_t* cached = nullptr;
+  for (int l = 0; l < n_layers; ++l) {
+    if (pattern[l] == 'F') {
+      int32_t* buf = f_bufs[n_fbufs == 1 ? 0 : m];
+      ++m;
+      const dsa_layer_inputs& in = layers[l];
+      dsa_status st;
+      if (shape->mode == DSA_MODE_PREFILL)
+        st = dsa_indexer_prefill(in.q, in.q_scale, in.w, in.k, in.k_scale, shape->Lk, shape->q_pos0,
+                                 shape->Lq, shape->H, shape->d, shape->topk, buf, in.out_score,
+                                 workspace, workspace_bytes, stream);
+      else
+        st = dsa_indexer_decode(in.q, in.q_scale, in.w, in.k, in.k_scale, shape->n_blocks,
+                                shape->block_size, shape->block_table, shape->max_blocks,
+                                shape->seq_lens, shape->B, shape->H, shape->d, shape->topk, buf,
+                                in.out_score, workspace, workspace_bytes, stream);
+      if (st != DSA_OK) return st;
+      cached = buf;
+    }
+    out_layer_idx[l] = cached;  // an S layer reads T_f(l): the buffer of the last F layer
+    if (after_layer) after_layer(l, cached, user);
+  }
+  return DSA_OK;
+}
+
+DSA_API dsa_status topk_overlap(const int32_t* const* layer_idx, int32_t n_layers, int32_t rows,
+                                int32_t topk, int32_t n_keys, uint64_t* out_counts,
+                                uint64_t* out_valid, double* out_overlap, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  if (!layer_idx || !out_counts || !out_valid || !workspace) return DSA_ERR_INVALID;
+  if (n_layers < 1 || n_layers > DSA_MAX_LAYERS || rows < 0 || topk < 1 || n_keys < 1)
+    return DSA_ERR_INVALID;
+  if (n_keys > 1500000) return DSA_ERR_UNSUPPORTED;
+  if (workspace_bytes < DSA_WS_HEADER_BYTES || !aligned(workspace, 256)) return DSA_ERR_INVALID;
+  for (int i = 0; i < n_layers; ++i)
+    if (!layer_idx[i]) return DSA_ERR_INVALID;
+  const int sms = current_num_sms();
+  if (sms < 1) return DSA_ERR_CUDA;
+  return launch_overlap(layer_idx, n_layers, rows, topk, n_keys, out_counts, out_valid, out_overlap,
+                        workspace, static_cast<cudaStream_t>(stream), sms);
+}
+
+DSA_API dsa_status dsa_selftest_wait_timeout(void* workspace, size_t workspace_bytes,
+                                             uint64_t budget_ns, void* stream) {
+  if (!workspace || workspace_bytes < DSA_WS_HEADER_BYTES || !aligned(workspace, 256) ||
+      budget_ns == 0 || budget_ns > 10000000000ull)
+    return DSA_ERR_INVALID;
+  return launch_selftest_wait(workspace, budget_ns, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,287 @@
+// Shared device helpers for the DSA indexer kernels (sm_100a only).
+//
+// PTX wrappers for mbarriers, TMA tile loads, tcgen05 (TMEM alloc, MMA, commit, loads),
+// bounded waits that record a timeout in the workspace header instead of spinning
+// forever, and the order-preserving 64-bit (score, index) key used by every top-k stage.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/dsa_indexer.h"
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "this library targets sm_100a only"
+#endif
+
+namespace dsa {
+
+// ------------------------------------------------------------------------------------------
+// Workspace header (first DSA_WS_HEADER_BYTES of every workspace).
+// ------------------------------------------------------------------------------------------
+struct WsHeader {
+  uint32_t status;   // first device-side error (dsa_status), 0 = none
+  uint32_t detail;   // error detail (which check, or which wait timed out)
+  uint32_t reserved[62];
+};
+static_assert(sizeof(WsHeader) == DSA_WS_HEADER_BYTES, "workspace header size");
+
+// Error details recorded with DSA_ERR_TIMEOUT / DSA_ERR_DEVICE.
+enum : uint32_t {
+  DETAIL_WAIT_KFULL = 1,
+  DETAIL_WAIT_KEMPTY = 2,
+  DETAIL_WAIT_QFULL = 3,
+  DETAIL_WAIT_QEMPTY = 4,
+  DETAIL_WAIT_ACCFULL = 5,
+  DETAIL_WAIT_ACCEMPTY = 6,
+  DETAIL_WAIT_DRAIN = 7,
+  DETAIL_WAIT_SELFTEST = 8,
+  DETAIL_BAD_BLOCK_TABLE = 16,
+  DETAIL_BAD_SEQ_LEN = 17,
+  DETAIL_BAD_INDEX = 18,
+};
+
+__device__ __forceinline__ void record_error(WsHeader* hdr, uint32_t status, uint32_t detail) {
+  if (atomicCAS(&hdr->status, 0u, status) == 0u) atomicExch(&hdr->detail, detail);
+}
+
+// ------------------------------------------------------------------------------------------
+// Small utilities.
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }
+
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
+// Named barrier over `count` threads (warp-aligned groups).
+__device__ __forceinline__ void named_bar(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Named barrier that also ANDs a predicate across the participating threads.
+__device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t count, bool pred) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %3, 0;\n\t"
+      "bar.red.and.pred po, %1, %2, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(out)
+      : "r"(id), "r"(count), "r"(pred ? 1u : 0u)
+      : "memory");
+  return out != 0;
+}
+
+// Order-preserving map of an fp32 score to uint32 (larger score -> larger key).
+__device__ __forceinline__ uint32_t float_to_ordered(float f) {
+  uint32_t u = __float_as_uint(f);
+  return u ^ ((u & 0x80000000u) ? 0xFFFFFFFFu : 0x80000000u);
+}
+__device__ __forceinline__ float ordered_to_float(uint32_t o) {
+  uint32_t u = o ^ ((o & 0x80000000u) ? 0x80000000u : 0xFFFFFFFFu);
+  return __uint_as_float(u);
+}
+// 64-bit selection key: larger key = better = (higher score, then lower index).
+// Key 0 is below every real key and marks an empty slot.
+__device__ __forceinline__ uint64_t make_key(float score, uint32_t idx) {
+  return (static_cast<uint64_t>(float_to_ordered(score + 0.0f)) << 32) |
+         static_cast<uint64_t>(0xFFFFFFFFu - idx);
+}
+__device__ __forceinline__ int32_t key_index(uint64_t key) {
+  return key ? static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(key)) : -1;
+}
+__device__ __forceinline__ float key_score(uint64_t key) {
+  return key ? ordered_to_float(static_cast<uint32_t>(key >> 32)) : -__int_as_float(0x7f800000);
+}
+
+// ------------------------------------------------------------------------------------------
+// mbarrier
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Control block shared by the warps of one CTA for bounded waits.
+struct WaitCtl {
+  WsHeader* hdr;          // global workspace header
+  volatile int* abort;    // CTA-wide abort flag in shared memory
+  uint64_t budget_ns;     // longest single wait before giving up
+};
+
+// Waits for the phase with the given parity to complete. Returns false (and raises the
+// CTA abort flag, recording DSA_ERR_TIMEOUT on the first failure) if the wait exceeds the
+// budget or another warp of the CTA already aborted.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtl& ctl,
+                                          uint32_t detail) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t start = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*ctl.abort) return false;
+    if (globaltimer_ns() - start > ctl.budget_ns) {
+      *ctl.abort = 1;
+      record_error(ctl.hdr, DSA_ERR_TIMEOUT, detail);
+      return false;
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// TMA (no multicast anywhere in this library)
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int32_t x,
+                                            int32_t y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ------------------------------------------------------------------------------------------
+// tcgen05
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+// Arrive on `bar` once all previously issued tcgen05.mma of this thread have completed.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+// D[tmem] (+)= A[smem] * B[smem]^T, FP8 E4M3 inputs (kind::f8f6f4), FP32 accumulate.
+__device__ __forceinline__ void tc_mma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+// Same wait, with the destination registers of the outstanding loads as read-write
+// operands so that the compiler cannot move their uses above the wait.
+__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+        "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+        "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),
+        "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),
+        "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+      :
+      : "memory");
+}
+
+// Bounded wait that ignores the abort flag: used to let this CTA's own asynchronous
+// copies and MMAs land before it exits. Returns false if the bound ran out.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity,
+                                                uint64_t budget_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t start = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - start > budget_ns) return false;
+  }
+  return true;
+}
+// 32 lanes x 32 consecutive 32-bit columns; thread i gets lane (taddr.lane + i).
+__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+// Shared-memory matrix descriptor for a K-major operand tile whose rows are `row_bytes`
+// (64 or 128) long, stored densely and swizzled to match the TMA load that wrote it
+// (SWIZZLE_64B / SWIZZLE_128B). The 8-row core-matrix groups are 8 * row_bytes apart.
+__device__ __forceinline__ uint64_t make_smem_desc(uint32_t smem_addr, uint32_t row_bytes) {
+  const uint64_t layout = (row_bytes == 128) ? 2ull : 4ull;  // SWIZZLE_128B : SWIZZLE_64B
+  uint64_t desc = 0;
+  desc |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);          // start address
+  desc |= static_cast<uint64_t>(1u) << 16;                              // leading byte offset (unused)
+  desc |= static_cast<uint64_t>(((8u * row_bytes) >> 4) & 0x3FFFu) << 32;  // stride byte offset
+  desc |= 1ull << 46;                                                   // descriptor version
+  desc |= layout << 61;
+  return desc;
+}
+
+// Instruction descriptor: E4M3 x E4M3 -> F32, both K-major, shape M x N.
+__host__ __device__ constexpr uint32_t make_idesc_f8(uint32_t M, uint32_t N) {
+  return (1u << 4)                 // D format F32
+         | (0u << 7) | (0u << 10)  // A, B format E4M3
+         | ((N >> 3) << 17)        // N / 8
+         | ((M >> 4) << 24);       // M / 16
+}
+
+}  // namespace dsa

@@ -1,0 +1,78 @@
+"""The C-ABI library loads without a GPU, exports every symbol include/*.h declares, and
+rejects malformed arguments on the host before touching CUDA."""
+
+import ctypes
+import glob
+import os
+import re
+import subprocess
+
+import pytest
+
+from sparse_attention_token_04_b200 import binding
+from sparse_attention_token_04_b200.build import LIB_PATH, ROOT, build
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(LIB_PATH):
+        build()
+    return binding.lib()
+
+
+def declared_functions():
+    names = []
+    for header in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(header).read()
+        names += re.findall(r"DSA_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for required in ("dsa_indexer_prefill", "dsa_indexer_decode", "indexcache_run", "topk_overlap"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert names
+    for name in names:
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", LIB_PATH], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert set(names) <= exported
+    # nothing else leaks out of the library's own code
+    assert not [s for s in exported if s.startswith("_ZN3dsa")]
+
+
+def test_status_strings_and_version(lib):
+    assert binding.dsa_abi_version() == 1
+    assert binding.status_string(0) == "ok"
+    assert "invalid" in binding.status_string(1)
+    assert binding.status_string(99) == "unknown status"
+
+
+def test_host_validation_without_gpu(lib):
+    nul = None
+    # null inputs
+    st = lib.dsa_indexer_prefill(nul, nul, nul, nul, nul, 16, 0, 16, 64, 128, 8, nul, nul, nul, 0, nul)
+    assert st == binding.DSA_ERR_INVALID
+    st = lib.dsa_indexer_decode(nul, nul, nul, nul, nul, 1, 64, nul, 1, nul, 1, 64, 128, 8, nul, nul,
+                                nul, 0, nul)
+    assert st == binding.DSA_ERR_INVALID
+    # patterns: leading S, bad character, wrong length
+    shape = binding.dsa_indexer_shape()
+    arr = (binding.dsa_layer_inputs * 2)()
+    fb = (ctypes.c_void_p * 1)(ctypes.c_void_p(16))
+    out = (ctypes.c_void_p * 2)()
+    for pat, n in ((b"SF", 2), (b"FX", 2), (b"FS", 3)):
+        st = lib.indexcache_run(pat, n, ctypes.byref(shape), arr, fb, 1, out, binding.AFTER_LAYER_FN(),
+                                None, None, 0, None)
+        assert st == binding.DSA_ERR_INVALID, pat
+    # overlap: too many layers / no pointers
+    ptrs = (ctypes.c_void_p * 1)()
+    assert lib.topk_overlap(ptrs, 65, 1, 1, 1, None, None, None, None, 0, None) == binding.DSA_ERR_INVALID
+    # unsupported head shape is reported before any launch
+    st = lib.dsa_prefill_workspace_bytes(16, 32, 128, 8)
+    assert st == 0
