@@ -129,6 +129,38 @@ DSA_API dsa_status dsa_indexer_decode(const uint8_t* q, const float* q_scale, co
                                       void* workspace, size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------------
+ * Decode indexer that allocates nothing (the pages have no counterpart to this entry point).
+ *
+ * For callers that cannot allocate device memory when they run the indexer: e.g. a plugin
+ * inside a host application whose allocator owns all device memory, or a decode loop that must
+ * not call cudaMalloc / cudaFree at step time (cudaFree synchronises the whole device). It
+ * computes exactly what dsa_indexer_decode computes, with the same arguments except that,
+ * instead of a workspace, its scratch is a fixed array inside the library:
+ * DSA_WS_HEADER_BYTES + DSA_NOALLOC_MAX_SCORES * 4 bytes (16 MiB + 256 B), held on every GPU
+ * that loads the library until the process exits.
+ *   - B * max_blocks * block_size must not exceed DSA_NOALLOC_MAX_SCORES; a larger call returns
+ *     DSA_ERR_UNSUPPORTED and enqueues nothing. Other errors are those of dsa_indexer_decode.
+ *   - device_status_out: optional DEVICE int32[2] that receives the call's device-side status
+ *     and detail (as dsa_read_device_status reports them); the fixed scratch's status is
+ *     cleared at the end of every call, so pass NULL only if those errors are not wanted.
+ *   - The first call on each device looks up the scratch's device address (cudaGetSymbolAddress)
+ *     with that device current and caches it; make that first call before any stream capture.
+ *   - Every call on a device shares the one scratch array and may leave data in it: calls whose
+ *     work overlaps on the GPU (other streams, other host threads) race and must be serialised
+ *     by the caller.
+ * -------------------------------------------------------------------------------------*/
+#define DSA_NOALLOC_MAX_SCORES 4194304
+
+DSA_API dsa_status dsa_indexer_decode_noalloc(const uint8_t* q, const float* q_scale, const float* w,
+                                              const uint8_t* k_cache, const float* k_scale_cache,
+                                              int32_t n_blocks, int32_t block_size,
+                                              const int32_t* block_table, int32_t max_blocks,
+                                              const int32_t* seq_lens, int32_t B, int32_t H,
+                                              int32_t d, int32_t topk, int32_t* out_idx,
+                                              float* out_score, int32_t* device_status_out,
+                                              void* stream);
+
+/* ---------------------------------------------------------------------------------------
  * IndexCache layer driver ("IndexShare deep-dive report" §2.1: Full layers run the indexer
  * and overwrite the cached indices, Shared layers take T <- T_f(l) with
  * f(l) = max{j < l : c_j = F}, the first layer is always F, and the cache costs no extra

@@ -63,6 +63,8 @@ _SIGNATURES = {
     "topk_overlap": (_i32, [ctypes.POINTER(_vp), _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp,
                             _sz, _vp]),
     "dsa_selftest_wait_timeout": (_i32, [_vp, _sz, _u64, _vp]),
+    "dsa_indexer_decode_noalloc": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _i32, _vp, _i32,
+                                          _i32, _i32, _i32, _vp, _vp, _vp, _vp]),
 }
 
 _LIB: Optional[ctypes.CDLL] = None
@@ -325,3 +327,35 @@ def topk_overlap_ptrs(ptrs: Sequence[int], rows: int, topk: int, n_keys: int, ou
 def dsa_selftest_wait_timeout(workspace: torch.Tensor, budget_ns: int, stream=None) -> None:
     _check(lib().dsa_selftest_wait_timeout(_ptr(workspace), workspace.numel(), int(budget_ns),
                                            _stream(stream)), "dsa_selftest_wait_timeout")
+
+
+DSA_NOALLOC_MAX_SCORES = 4194304
+
+
+def dsa_indexer_decode_noalloc(q, q_scale, w, k_cache, k_scale_cache, block_table, seq_lens,
+                               topk: int, out_idx, out_score=None, device_status=None, stream=None):
+    """Decode indexer that allocates no device memory: for callers that must not allocate at
+    step time. Outputs (and the optional device int32[2] status) are passed in by the caller;
+    the library's fixed scratch bounds B * max_blocks * block_size by DSA_NOALLOC_MAX_SCORES."""
+    B, H, d = (int(x) for x in q.shape)
+    n_blocks, block_size = int(k_cache.shape[0]), int(k_cache.shape[1])
+    max_blocks = int(block_table.shape[1])
+    _need(q, "q", torch.uint8)
+    _need(q_scale, "q_scale", torch.float32, (B,))
+    _need(w, "w", torch.float32, (B, H))
+    _need(k_cache, "k_cache", torch.uint8, (n_blocks, block_size, d))
+    _need(k_scale_cache, "k_scale_cache", torch.float32, (n_blocks, block_size))
+    _need(block_table, "block_table", torch.int32, (B, max_blocks))
+    _need(seq_lens, "seq_lens", torch.int32, (B,))
+    _need(out_idx, "out_idx", torch.int32, (B, topk))
+    if out_score is not None:
+        _need(out_score, "out_score", torch.float32, (B, topk))
+    if device_status is not None:
+        _need(device_status, "device_status", torch.int32, (2,))
+    _check(lib().dsa_indexer_decode_noalloc(_ptr(q), _ptr(q_scale), _ptr(w), _ptr(k_cache),
+                                            _ptr(k_scale_cache), n_blocks, block_size,
+                                            _ptr(block_table), max_blocks, _ptr(seq_lens), B, H, d,
+                                            topk, _ptr(out_idx), _ptr(out_score),
+                                            _ptr(device_status), _stream(stream)),
+           "dsa_indexer_decode_noalloc")
+    return out_idx, out_score
