@@ -136,10 +136,11 @@ DSA_API dsa_status dsa_indexer_decode(const uint8_t* q, const float* q_scale, co
  * not call cudaMalloc / cudaFree at step time (cudaFree synchronises the whole device). It
  * computes exactly what dsa_indexer_decode computes, with the same arguments except that,
  * instead of a workspace, its scratch is a fixed array inside the library:
- * DSA_WS_HEADER_BYTES + DSA_NOALLOC_MAX_SCORES * 4 bytes (16 MiB + 256 B), held on every GPU
- * that loads the library until the process exits.
- *   - B * max_blocks * block_size must not exceed DSA_NOALLOC_MAX_SCORES; a larger call returns
- *     DSA_ERR_UNSUPPORTED and enqueues nothing. Other errors are those of dsa_indexer_decode.
+ * DSA_WS_HEADER_BYTES + DSA_NOALLOC_MAX_SCORES * 4 + DSA_NOALLOC_MAX_REQUESTS * 8192 bytes
+ * (18 MiB + 256 B), held on every GPU that loads the library until the process exits.
+ *   - B must not exceed DSA_NOALLOC_MAX_REQUESTS and B * max_blocks * block_size must not exceed
+ *     DSA_NOALLOC_MAX_SCORES; a larger call returns DSA_ERR_UNSUPPORTED and enqueues nothing.
+ *     Other errors are those of dsa_indexer_decode.
  *   - device_status_out: optional DEVICE int32[2] that receives the call's device-side status
  *     and detail (as dsa_read_device_status reports them); the fixed scratch's status is
  *     cleared at the end of every call, so pass NULL only if those errors are not wanted.
@@ -150,6 +151,7 @@ DSA_API dsa_status dsa_indexer_decode(const uint8_t* q, const float* q_scale, co
  *     by the caller.
  * -------------------------------------------------------------------------------------*/
 #define DSA_NOALLOC_MAX_SCORES 4194304
+#define DSA_NOALLOC_MAX_REQUESTS 256
 
 DSA_API dsa_status dsa_indexer_decode_noalloc(const uint8_t* q, const float* q_scale, const float* w,
                                               const uint8_t* k_cache, const float* k_scale_cache,

@@ -40,6 +40,7 @@ enum : uint32_t {
   DETAIL_BAD_BLOCK_TABLE = 16,
   DETAIL_BAD_SEQ_LEN = 17,
   DETAIL_BAD_INDEX = 18,
+  DETAIL_HIST_MISMATCH = 19,
 };
 
 __device__ __forceinline__ void record_error(WsHeader* hdr, uint32_t status, uint32_t detail) {

@@ -10,19 +10,22 @@
 //   warp 1     one thread issues tcgen05.mma kind::f8f6f4, M = 128 keys, N = 64 heads,
 //              K = d, into one of two 64-column TMEM accumulators;
 //   warps 2-5  epilogue: thread = key; ReLU (on the FMA pipe, see prefill.cu), head weights,
-//              scales; the score of every valid key is stored at scores[b][s].
+//              scales; the score of every valid key is stored at scores[b][s] and counted in
+//              the request's histogram of order-preserving top-11-bit bins.
 // decode_topk_kernel (topk.cu) then selects and orders each request's top-k.
 #include "common.cuh"
 #include "internal.h"
 
 namespace dsa {
 
+constexpr int kScoreBins = 2048;  // bins of the top 11 bits of an order-preserving fp32 key
+
 template <int D>
 struct DCfg {
   static constexpr int H = 64;
   static constexpr int PAGE = 64;              // keys per cache block
   static constexpr int BN = 128;               // keys per tile
-  static constexpr int STAGES = 4;
+  static constexpr int STAGES = 3;
   static constexpr int TPC = 8;                // tiles per CTA
   static constexpr int QTILE = H * D;
   static constexpr int KTILE = BN * D;
@@ -38,6 +41,7 @@ struct DSmem {
   uint8_t q[C::QTILE];
   uint8_t k[C::STAGES][C::KTILE];
   float wq[C::H];
+  uint32_t hist[kScoreBins];   // this CTA's scores per order-preserving top-11-bit bin
   uint64_t kfull[C::STAGES];
   uint64_t kempty[C::STAGES];
   uint64_t qfull, accfull[2], accempty[2], drain;
@@ -53,6 +57,7 @@ struct DecodeParams {
   const int32_t* seq_lens;
   int32_t max_blocks, n_blocks, max_len;
   float* scores;
+  uint32_t* bins;   // [B][kScoreBins] per-request score histogram
   WsHeader* hdr;
   uint64_t budget_ns;
 };
@@ -171,6 +176,7 @@ __global__ void __launch_bounds__(192)
     const uint32_t wl = warp & 3u;
     const uint32_t rank = threadIdx.x - 64u;
     if (rank < C::H) sm.wq[rank] = __ldg(&p.w[static_cast<size_t>(b) * C::H + rank]) * 0x1p25f;
+    for (int i = rank; i < kScoreBins; i += 128) sm.hist[i] = 0u;
     named_bar(1, 128);
     const float sq = __ldg(&p.q_scale[b]);
     float* out = p.scores + static_cast<size_t>(b) * p.max_len;
@@ -213,8 +219,18 @@ __global__ void __launch_bounds__(192)
         part[3] = fmaf(w1.w, __saturatef(__uint_as_float(rb[j + 3]) * 0x1p-25f), part[3]);
       }
       const float acc = (part[0] + part[1]) + (part[2] + part[3]);
-      if (valid && got) out[s] = (acc * sq) * sk;
+      if (valid && got) {
+        const float score = (acc * sq) * sk;
+        out[s] = score;
+        atomicAdd(&sm.hist[float_to_ordered(score + 0.0f) >> 21], 1u);
+      }
       if (!__all_sync(0xFFFFFFFFu, got)) break;
+    }
+    named_bar(1, 128);
+    uint32_t* gbins = p.bins + static_cast<size_t>(b) * kScoreBins;
+    for (int i = rank; i < kScoreBins; i += 128) {
+      const uint32_t c = sm.hist[i];
+      if (c) atomicAdd(&gbins[i], c);
     }
   }
   __syncthreads();
@@ -249,20 +265,26 @@ static dsa_status launch_decode_t(const DecodeLaunch& a) {
   uint8_t* base = static_cast<uint8_t*>(a.ws);
   p.hdr = reinterpret_cast<WsHeader*>(base);
   p.scores = reinterpret_cast<float*>(base + DSA_WS_HEADER_BYTES);
+  p.bins = reinterpret_cast<uint32_t*>(base + DSA_WS_HEADER_BYTES +
+                                       static_cast<size_t>(a.B) * max_len * sizeof(float));
   p.budget_ns = a.budget_ns;
+  if (cudaMemsetAsync(p.bins, 0, static_cast<size_t>(a.B) * kScoreBins * sizeof(uint32_t), a.stream) !=
+      cudaSuccess)
+    return DSA_ERR_CUDA;
   const int max_tiles = (max_len + C::BN - 1) / C::BN;
   dim3 grid((max_tiles + C::TPC - 1) / C::TPC, a.B);
   kern<<<grid, C::THREADS, smem, a.stream>>>(tq, tk, p);
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
-  return launch_decode_topk(p.scores, max_len, a.seq_lens, a.B, a.topk, a.out_idx, a.out_score,
-                            a.ws, a.stream);
+  return launch_decode_topk(p.scores, max_len, a.seq_lens, p.bins, a.B, a.topk, a.out_idx,
+                            a.out_score, a.ws, a.stream);
 }
 
 size_t decode_workspace_bytes(int B, int max_len, int H, int d, int topk) {
   (void)H;
   (void)d;
   (void)topk;
-  return DSA_WS_HEADER_BYTES + static_cast<size_t>(B) * max_len * sizeof(float);
+  return DSA_WS_HEADER_BYTES + static_cast<size_t>(B) * max_len * sizeof(float) +
+         static_cast<size_t>(B) * kScoreBins * sizeof(uint32_t);
 }
 
 dsa_status launch_decode(const DecodeLaunch& a) {

@@ -60,9 +60,9 @@ dsa_status launch_prefill(const PrefillLaunch& a);
 dsa_status launch_decode(const DecodeLaunch& a);
 dsa_status launch_sort_rows(const uint64_t* win, int rows, int topk, int32_t* out_idx,
                             float* out_score, cudaStream_t stream);
-dsa_status launch_decode_topk(const float* scores, int max_len, const int32_t* seq_lens, int B,
-                              int topk, int32_t* out_idx, float* out_score, void* ws,
-                              cudaStream_t stream);
+dsa_status launch_decode_topk(const float* scores, int max_len, const int32_t* seq_lens,
+                              const uint32_t* bins, int B, int topk, int32_t* out_idx,
+                              float* out_score, void* ws, cudaStream_t stream);
 dsa_status launch_overlap(const int32_t* const* layer_idx, int32_t n_layers, int32_t rows,
                           int32_t topk, int32_t n_keys, uint64_t* out_counts, uint64_t* out_valid,
                           double* out_overlap, void* ws, cudaStream_t stream, int num_sms);

@@ -20,11 +20,13 @@
 namespace dsa {
 namespace {
 
-constexpr size_t kScratchBytes =
-    DSA_WS_HEADER_BYTES + static_cast<size_t>(DSA_NOALLOC_MAX_SCORES) * sizeof(float);
+// Status header, one fp32 score slot per cached key, and a 2048-bin score histogram per request.
+constexpr size_t kScratchBytes = DSA_WS_HEADER_BYTES +
+                                 static_cast<size_t>(DSA_NOALLOC_MAX_SCORES) * sizeof(float) +
+                                 static_cast<size_t>(DSA_NOALLOC_MAX_REQUESTS) * 2048 * sizeof(uint32_t);
 
-// Status header followed by the score slots. Zero at load time; the header is cleared again at
-// the end of every call, so each call starts with a clean status.
+// Zero at load time; the status header is cleared again at the end of every call, so each call
+// starts with a clean status (the decode launch itself clears the histograms it uses).
 static __device__ __align__(256) uint8_t g_decode_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
@@ -57,8 +59,10 @@ extern "C" DSA_API dsa_status dsa_indexer_decode_noalloc(
     int32_t* out_idx, float* out_score, int32_t* device_status_out, void* stream) {
   using namespace dsa;
   if (B >= 1 && max_blocks >= 1 && block_size >= 1 &&
-      static_cast<int64_t>(B) * max_blocks * block_size > static_cast<int64_t>(DSA_NOALLOC_MAX_SCORES))
-    return DSA_ERR_UNSUPPORTED;  // more cached-key slots than the fixed scratch holds
+      (B > DSA_NOALLOC_MAX_REQUESTS ||
+       static_cast<int64_t>(B) * max_blocks * block_size > static_cast<int64_t>(DSA_NOALLOC_MAX_SCORES) ||
+       dsa_decode_workspace_bytes(B, max_blocks * block_size, H, d, topk) > kScratchBytes))
+    return DSA_ERR_UNSUPPORTED;  // more requests or cached-key slots than the fixed scratch holds
   void* scratch = nullptr;
   dsa_status st = scratch_address(&scratch);
   if (st != DSA_OK) return st;

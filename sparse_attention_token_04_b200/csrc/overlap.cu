@@ -1,10 +1,12 @@
 // Cross-layer top-k overlap: C[i][j] = sum over rows of |T_i(row) ∩ T_j(row)|.
 //
-// Integer work bound by reading the N index tensors (N * rows * topk * 4 bytes). Each CTA
-// walks rows; for a row and each layer i it marks T_i(row) in a shared-memory bitmap over
-// [0, n_keys), probes the entries of T_j(row), j >= i, against it, and clears the marked
-// words again. Counts accumulate in shared 64-bit counters per CTA and are added to the
-// output once per CTA. A finishing kernel mirrors the upper triangle and forms C / V.
+// Integer work bound by reading the N index tensors (N * rows * topk * 4 bytes, each byte once).
+// A CTA walks rows. For a row it marks every layer's indices in per-layer shared-memory bitmaps
+// over the row's index range, counts each pair (i <= j) as the popcount of the AND of the two
+// bitmaps, and clears the bitmaps. When the N bitmaps over [0, n_keys) do not fit in shared
+// memory, one bitmap at a time is built and the other layers' entries are probed against it.
+// Counts accumulate in shared 64-bit counters per CTA and are added to the output once per CTA;
+// a finishing kernel mirrors the upper triangle and forms C / V.
 #include "common.cuh"
 #include "internal.h"
 
@@ -19,13 +21,83 @@ struct OverlapParams {
 };
 
 constexpr int kOverlapThreads = 256;
+constexpr size_t kOverlapSmemBudget = 200 * 1024;
 
+__device__ __forceinline__ unsigned long long* overlap_acc(uint8_t* smem) {
+  return reinterpret_cast<unsigned long long*>(smem);
+}
+
+// All N bitmaps resident: bits[i][w], W words per layer.
 __global__ void __launch_bounds__(kOverlapThreads)
-    overlap_kernel(const __grid_constant__ OverlapParams p) {
-  extern __shared__ uint8_t smem_raw[];
+    overlap_bitmaps_kernel(const __grid_constant__ OverlapParams p) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
   const int N = p.N;
-  unsigned long long* acc = reinterpret_cast<unsigned long long*>(smem_raw);     // [N*N + 1]
-  uint32_t* bits = reinterpret_cast<uint32_t*>(acc + (N * N + 1));               // [W]
+  const int npairs = N * (N + 1) / 2;
+  unsigned long long* acc = overlap_acc(smem_raw);                        // [npairs + 1]
+  int* row_max = reinterpret_cast<int*>(acc + npairs + 1);                 // [1] (+pad)
+  uint32_t* bits = reinterpret_cast<uint32_t*>(row_max + 4);               // [N][W]
+  const int W = (p.n_keys + 31) / 32;
+  for (int e = threadIdx.x; e < npairs + 1; e += kOverlapThreads) acc[e] = 0ull;
+  for (int e = threadIdx.x; e < N * W; e += kOverlapThreads) bits[e] = 0u;
+  if (threadIdx.x == 0) *row_max = -1;
+  __syncthreads();
+  const uint32_t lane = threadIdx.x & 31u;
+  for (int row = blockIdx.x; row < p.rows; row += gridDim.x) {
+    const size_t off = static_cast<size_t>(row) * p.topk;
+    int local_max = -1;
+    uint32_t valid0 = 0;
+    for (int i = 0; i < N; ++i) {
+      const int32_t* Ti = p.layers[i] + off;
+      uint32_t* bi = bits + i * W;
+      for (int e = threadIdx.x; e < p.topk; e += kOverlapThreads) {
+        const int32_t v = __ldcs(&Ti[e]);
+        if (v >= 0 && v < p.n_keys) {
+          atomicOr(&bi[v >> 5], 1u << (v & 31));
+          local_max = v > local_max ? v : local_max;
+          if (i == 0) ++valid0;
+        } else if (v != -1) {
+          record_error(p.hdr, DSA_ERR_DEVICE, DETAIL_BAD_INDEX);
+        }
+      }
+    }
+    if (local_max >= 0) atomicMax(row_max, local_max);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) valid0 += __shfl_xor_sync(0xFFFFFFFFu, valid0, o);
+    if (lane == 0 && valid0) atomicAdd(&acc[npairs], static_cast<unsigned long long>(valid0));
+    __syncthreads();
+    const int wr = (*row_max >> 5) + 1;  // words that can hold a mark in this row
+    int pair = 0;
+    for (int i = 0; i < N; ++i) {
+      const uint32_t* bi = bits + i * W;
+      for (int j = i; j < N; ++j, ++pair) {
+        const uint32_t* bj = bits + j * W;
+        uint32_t c = 0;
+        for (int w = threadIdx.x; w < wr; w += kOverlapThreads) c += __popc(bi[w] & bj[w]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xFFFFFFFFu, c, o);
+        if (lane == 0 && c) atomicAdd(&acc[pair], static_cast<unsigned long long>(c));
+      }
+    }
+    __syncthreads();
+    for (int i = 0; i < N; ++i)
+      for (int w = threadIdx.x; w < wr; w += kOverlapThreads) bits[i * W + w] = 0u;
+    if (threadIdx.x == 0) *row_max = -1;
+    __syncthreads();
+  }
+  int pair = 0;
+  for (int i = 0; i < N; ++i)
+    for (int j = i; j < N; ++j, ++pair)
+      if (threadIdx.x == 0 && acc[pair]) atomicAdd(&p.counts[i * N + j], acc[pair]);
+  if (threadIdx.x == 0 && acc[npairs]) atomicAdd(p.valid, acc[npairs]);
+}
+
+// One bitmap at a time (wide index ranges or many layers).
+__global__ void __launch_bounds__(kOverlapThreads)
+    overlap_probe_kernel(const __grid_constant__ OverlapParams p) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  const int N = p.N;
+  unsigned long long* acc = overlap_acc(smem_raw);                        // [N*N + 1]
+  uint32_t* bits = reinterpret_cast<uint32_t*>(acc + (N * N + 1));        // [W]
   const int W = (p.n_keys + 31) / 32;
   for (int e = threadIdx.x; e < N * N + 1; e += kOverlapThreads) acc[e] = 0ull;
   for (int e = threadIdx.x; e < W; e += kOverlapThreads) bits[e] = 0u;
@@ -37,11 +109,8 @@ __global__ void __launch_bounds__(kOverlapThreads)
       const int32_t* Ti = p.layers[i] + off;
       for (int e = threadIdx.x; e < p.topk; e += kOverlapThreads) {
         const int32_t v = __ldg(&Ti[e]);
-        if (v >= 0 && v < p.n_keys) {
-          atomicOr(&bits[v >> 5], 1u << (v & 31));
-        } else if (v != -1) {
-          record_error(p.hdr, DSA_ERR_DEVICE, DETAIL_BAD_INDEX);
-        }
+        if (v >= 0 && v < p.n_keys) atomicOr(&bits[v >> 5], 1u << (v & 31));
+        else if (v != -1) record_error(p.hdr, DSA_ERR_DEVICE, DETAIL_BAD_INDEX);
       }
       __syncthreads();
       for (int j = i; j < N; ++j) {
@@ -88,6 +157,21 @@ __global__ void overlap_finish_kernel(unsigned long long* counts, const unsigned
   }
 }
 
+template <class Kern>
+static dsa_status launch_overlap_kernel(Kern kern, const OverlapParams& p, size_t smem, int rows,
+                                        cudaStream_t stream, int num_sms) {
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kOverlapThreads, smem) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  if (per_sm < 1) return DSA_ERR_UNSUPPORTED;
+  const int grid = rows < per_sm * num_sms ? rows : per_sm * num_sms;
+  kern<<<grid, kOverlapThreads, smem, stream>>>(p);
+  return cuda_status(cudaGetLastError());
+}
+
 dsa_status launch_overlap(const int32_t* const* layer_idx, int32_t n_layers, int32_t rows,
                           int32_t topk, int32_t n_keys, uint64_t* out_counts, uint64_t* out_valid,
                           double* out_overlap, void* ws, cudaStream_t stream, int num_sms) {
@@ -104,18 +188,16 @@ dsa_status launch_overlap(const int32_t* const* layer_idx, int32_t n_layers, int
   if (cudaMemsetAsync(out_counts, 0, nn * sizeof(uint64_t), stream) != cudaSuccess) return DSA_ERR_CUDA;
   if (cudaMemsetAsync(out_valid, 0, sizeof(uint64_t), stream) != cudaSuccess) return DSA_ERR_CUDA;
   if (rows > 0) {
-    const size_t smem = (nn + 1) * sizeof(unsigned long long) + static_cast<size_t>((n_keys + 31) / 32) * 4;
-    if (cudaFuncSetAttribute(overlap_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return DSA_ERR_CUDA;
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, overlap_kernel, kOverlapThreads, smem) !=
-        cudaSuccess)
-      return DSA_ERR_CUDA;
-    if (per_sm < 1) return DSA_ERR_UNSUPPORTED;
-    const int grid = rows < per_sm * num_sms ? rows : per_sm * num_sms;
-    overlap_kernel<<<grid, kOverlapThreads, smem, stream>>>(p);
-    if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+    const size_t words = static_cast<size_t>((n_keys + 31) / 32);
+    const size_t npairs = static_cast<size_t>(n_layers) * (n_layers + 1) / 2;
+    const size_t smem_all = (npairs + 1) * 8 + 16 + static_cast<size_t>(n_layers) * words * 4;
+    dsa_status st;
+    if (smem_all <= kOverlapSmemBudget)
+      st = launch_overlap_kernel(overlap_bitmaps_kernel, p, smem_all, rows, stream, num_sms);
+    else
+      st = launch_overlap_kernel(overlap_probe_kernel, p, (nn + 1) * 8 + words * 4, rows, stream,
+                                 num_sms);
+    if (st != DSA_OK) return st;
   }
   overlap_finish_kernel<<<1, 256, 0, stream>>>(p.counts, p.valid, out_overlap, n_layers);
   return cuda_status(cudaGetLastError());

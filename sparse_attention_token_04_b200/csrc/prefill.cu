@@ -11,8 +11,9 @@
 //               it reads the key's H head dot products of each query, applies
 //               ReLU, the head weights, then the query and key scales, masks s > t, and
 //               streams keys that can still enter the top-k into a per-query candidate
-//               buffer (workspace). A full buffer is cut back to exactly topk keys by an
-//               exact radix select, which also raises the query's insertion threshold.
+//               buffer (workspace). A nearly full buffer is staged in shared memory and cut
+//               back to exactly topk keys by an exact radix select, which also raises the
+//               query's insertion threshold.
 // After the last tile every query's buffer is reduced to exactly its top-k keys and written
 // to the winners array; the row sort (topk.cu) orders them. The L x L score matrix is never
 // stored.
@@ -42,6 +43,8 @@ struct PCfg {
   static_assert(H == 8 || H == 64, "H");
 };
 
+constexpr int kCandCapMax = 2 * DSA_MAX_TOPK + 256;
+
 template <int H, int D>
 struct PSmem {
   using C = PCfg<H, D>;
@@ -51,15 +54,30 @@ struct PSmem {
   float sq[C::QB];
   uint64_t thr[C::QB];
   uint32_t cnt[C::QB];
-  uint32_t cur[C::QB];
   uint32_t hist[2][kHistBins];
-  uint32_t scratch[2][8];
+  GroupScratch<128> gsc[2];
+  uint64_t stage[2][kCandCapMax];   // a candidate buffer staged for a cut-back
   uint64_t kfull[C::STAGES];
   uint64_t kempty[C::STAGES];
   uint64_t qfull, qempty, accfull[2], accempty[2], drain;
   uint32_t tmem_base;
   int abort;
 };
+
+// Copies n candidate keys from global memory into shared memory, eight independent loads in
+// flight per thread.
+__device__ __forceinline__ void stage_keys(const uint64_t* __restrict__ src, uint32_t n,
+                                           uint64_t* __restrict__ dst, uint32_t rank) {
+  uint32_t e = rank;
+  for (; e + 7 * 128 < n; e += 8 * 128) {
+    uint64_t v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __ldcg(src + e + i * 128);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) dst[e + i * 128] = v[i];
+  }
+  for (; e < n; e += 128) dst[e] = __ldcg(src + e);
+}
 
 struct PrefillParams {
   const float* q_scale;
@@ -119,8 +137,8 @@ __global__ void __launch_bounds__(384, 1)
     const int last_row = min(qb * C::QB + C::QB, p.Lq) - 1;
     return (p.q_pos0 + last_row) / C::BN + 1;
   };
-  auto cand_buf = [&](int qidx, uint32_t which) -> uint64_t* {
-    return p.cand + ((static_cast<size_t>(cta) * C::QB + qidx) * 2 + which) * p.cap;
+  auto cand_buf = [&](int qidx) -> uint64_t* {
+    return p.cand + (static_cast<size_t>(cta) * C::QB + qidx) * p.cap;
   };
 
   if (warp == 0) {
@@ -215,7 +233,8 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t rank = threadIdx.x - 128u * (1u + g);
     const GroupSync<128> gs{1u + g};
     uint32_t* hist = sm.hist[g];
-    uint32_t* scr = sm.scratch[g];
+    GroupScratch<128>& scr = sm.gsc[g];
+    uint64_t* stage = sm.stage[g];
     const uint32_t taddr0 = tmem + g * 256 + ((wl * 32u) << 16);
     const int qbase = static_cast<int>(g) * C::QPM;
     uint32_t use = 0;
@@ -234,7 +253,6 @@ __global__ void __launch_bounds__(384, 1)
         sm.sq[qbase + qi] = (row < p.Lq) ? __ldg(&p.q_scale[row]) : 0.0f;
         sm.thr[qbase + qi] = 0;
         sm.cnt[qbase + qi] = 0;
-        sm.cur[qbase + qi] = 0;
       }
       gs.sync();
       const int nt = ntiles_of(qb);
@@ -289,29 +307,28 @@ __global__ void __launch_bounds__(384, 1)
             uint32_t base = 0;
             if (lane == 0) base = atomicAdd(&sm.cnt[qbase + qi], static_cast<uint32_t>(__popc(m)));
             base = __shfl_sync(0xFFFFFFFFu, base, 0);
-            if (take)
-              cand_buf(qbase + qi, sm.cur[qbase + qi])[base + __popc(m & ((1u << lane) - 1u))] = key;
+            if (take) cand_buf(qbase + qi)[base + __popc(m & ((1u << lane) - 1u))] = key;
           }
         }
         ok = named_bar_and(1u + g, 128, ok && got);
         if (!ok) break;
-        // Cut any nearly full candidate buffer back to exactly topk keys.
+        // Cut any nearly full candidate buffer back to exactly topk keys: stage it in shared
+        // memory, find the threshold there, write the survivors back to the buffer's front.
         for (int qi = 0; qi < C::QPM; ++qi) {
           const uint32_t n = sm.cnt[qbase + qi];
           if (n <= p.cap - 128u) continue;
-          const uint32_t which = sm.cur[qbase + qi];
-          const uint64_t* src = cand_buf(qbase + qi, which);
-          uint64_t* dst = cand_buf(qbase + qi, which ^ 1u);
-          auto key_at = [&](uint32_t e) { return src[e]; };
-          const uint64_t T = group_kth_threshold<128>(key_at, n, static_cast<uint32_t>(p.topk),
-                                                      rank, hist, scr, gs);
-          group_compact_ge<128>(key_at, n, T, [&](uint32_t pos, uint64_t key) { if (pos < p.cap) dst[pos] = key; },
-                                rank, scr, gs);
+          uint64_t* buf = cand_buf(qbase + qi);
+          stage_keys(buf, n, stage, rank);
           gs.sync();
+          auto key_at = [&](uint32_t e) { return stage[e]; };
+          const uint32_t k = static_cast<uint32_t>(p.topk);
+          const uint64_t T = group_kth_threshold<128>(key_at, n, k, rank, hist, scr, gs);
+          group_compact_ge<128>(key_at, n, T,
+                                [&](uint32_t pos, uint64_t key) { if (pos < k) buf[pos] = key; },
+                                rank, scr, gs);
           if (rank == 0) {
             sm.thr[qbase + qi] = T;
-            sm.cnt[qbase + qi] = static_cast<uint32_t>(p.topk);
-            sm.cur[qbase + qi] = which ^ 1u;
+            sm.cnt[qbase + qi] = k;
           }
           gs.sync();
         }
@@ -322,18 +339,19 @@ __global__ void __launch_bounds__(384, 1)
         const int row = row_base + qi;
         if (row >= p.Lq) break;
         const uint32_t n = sm.cnt[qbase + qi];
-        const uint64_t* src = cand_buf(qbase + qi, sm.cur[qbase + qi]);
+        const uint32_t k = static_cast<uint32_t>(p.topk);
+        const uint64_t* buf = cand_buf(qbase + qi);
         uint64_t* dst = p.win + static_cast<size_t>(row) * p.topk;
-        if (n > static_cast<uint32_t>(p.topk)) {
-          auto key_at = [&](uint32_t e) { return src[e]; };
-          const uint64_t T = group_kth_threshold<128>(key_at, n, static_cast<uint32_t>(p.topk),
-                                                      rank, hist, scr, gs);
+        if (n > k) {
+          stage_keys(buf, n, stage, rank);
+          gs.sync();
+          auto key_at = [&](uint32_t e) { return stage[e]; };
+          const uint64_t T = group_kth_threshold<128>(key_at, n, k, rank, hist, scr, gs);
           group_compact_ge<128>(key_at, n, T,
-                                [&](uint32_t pos, uint64_t key) { if (pos < static_cast<uint32_t>(p.topk)) dst[pos] = key; },
+                                [&](uint32_t pos, uint64_t key) { if (pos < k) dst[pos] = key; },
                                 rank, scr, gs);
         } else {
-          for (uint32_t e = rank; e < static_cast<uint32_t>(p.topk); e += 128)
-            dst[e] = (e < n) ? src[e] : 0ull;
+          for (uint32_t e = rank; e < k; e += 128) dst[e] = (e < n) ? buf[e] : 0ull;
         }
         gs.sync();
       }
@@ -376,7 +394,7 @@ static dsa_status launch_prefill_t(const PrefillLaunch& a) {
   p.cap = prefill_cand_cap(a.topk);
   p.hdr = reinterpret_cast<WsHeader*>(base);
   p.cand = reinterpret_cast<uint64_t*>(base + DSA_WS_HEADER_BYTES);
-  const size_t cand_bytes = static_cast<size_t>(a.num_sms) * C::QB * 2 * p.cap * sizeof(uint64_t);
+  const size_t cand_bytes = static_cast<size_t>(a.num_sms) * C::QB * p.cap * sizeof(uint64_t);
   p.win = reinterpret_cast<uint64_t*>(base + DSA_WS_HEADER_BYTES + cand_bytes);
   p.budget_ns = a.budget_ns;
   kern<<<grid, C::THREADS, smem, a.stream>>>(tq, tk, p);
@@ -387,7 +405,7 @@ static dsa_status launch_prefill_t(const PrefillLaunch& a) {
 size_t prefill_workspace_bytes(int Lq, int H, int d, int topk, int num_sms) {
   (void)d;
   const size_t qb = static_cast<size_t>(prefill_queries_per_block(H));
-  const size_t cand = static_cast<size_t>(num_sms) * qb * 2 * prefill_cand_cap(topk) * sizeof(uint64_t);
+  const size_t cand = static_cast<size_t>(num_sms) * qb * prefill_cand_cap(topk) * sizeof(uint64_t);
   const size_t win = static_cast<size_t>(Lq) * topk * sizeof(uint64_t);
   return DSA_WS_HEADER_BYTES + cand + win;
 }

@@ -8,18 +8,7 @@
 
 namespace dsa {
 
-constexpr int kHistBins = 2048;  // 11-bit radix digits
-
-// Digits of the 64-bit key, most significant first: the score word in 11/11/10 bits, then
-// the index word in 11/11/10 bits.
-__device__ __forceinline__ int radix_shift(int pass) {
-  constexpr int s[6] = {53, 42, 32, 21, 10, 0};
-  return s[pass];
-}
-__device__ __forceinline__ int radix_bits(int pass) {
-  constexpr int b[6] = {11, 11, 10, 11, 11, 10};
-  return b[pass];
-}
+constexpr int kHistBins = 2048;  // radix digits of up to 11 bits
 
 template <int NT>
 struct GroupSync {
@@ -27,8 +16,15 @@ struct GroupSync {
   __device__ __forceinline__ void sync() const { named_bar(bar_id, NT); }
 };
 
+// Scratch words a group needs: NT/32 + 2 (u32) and 2 * NT/32 (u64).
+template <int NT>
+struct GroupScratch {
+  uint32_t w[NT / 32 + 2];
+  uint64_t w64[2 * (NT / 32)];
+};
+
 // Sum of `v` over the threads of the group whose rank is HIGHER than this thread's
-// (exclusive suffix sum), and the group total. `scratch` holds NT/32 words.
+// (exclusive suffix sum), and the group total.
 template <int NT>
 __device__ __forceinline__ uint32_t group_suffix_exclusive(uint32_t v, uint32_t rank,
                                                            uint32_t* scratch,
@@ -84,20 +80,62 @@ __device__ __forceinline__ uint32_t group_prefix_exclusive(uint32_t v, uint32_t 
   return below + (s - v);
 }
 
-// Returns T such that exactly k of the n keys produced by key_at(e), e in [0, n), satisfy
-// key >= T. Requires 0 < k < n and distinct keys. `hist` holds kHistBins words and
-// `scratch` at least NT/32 + 2 words, both private to the group.
+// Smallest and largest of the n keys key_at(e), over the group.
+template <int NT, class KeyAt>
+__device__ void group_minmax(KeyAt key_at, uint32_t n, uint32_t rank, GroupScratch<NT>& sc,
+                             const GroupSync<NT>& gs, uint64_t* mn, uint64_t* mx) {
+  constexpr int NW = NT / 32;
+  uint64_t lo = ~0ull, hi = 0ull;
+  for (uint32_t e = rank; e < n; e += NT) {
+    const uint64_t v = key_at(e);
+    lo = v < lo ? v : lo;
+    hi = v > hi ? v : hi;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const uint64_t a = __shfl_xor_sync(0xFFFFFFFFu, lo, off);
+    const uint64_t b = __shfl_xor_sync(0xFFFFFFFFu, hi, off);
+    lo = a < lo ? a : lo;
+    hi = b > hi ? b : hi;
+  }
+  if ((rank & 31u) == 0) {
+    sc.w64[2 * (rank >> 5)] = lo;
+    sc.w64[2 * (rank >> 5) + 1] = hi;
+  }
+  gs.sync();
+  lo = ~0ull;
+  hi = 0ull;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) {
+    const uint64_t a = sc.w64[2 * w], b = sc.w64[2 * w + 1];
+    lo = a < lo ? a : lo;
+    hi = b > hi ? b : hi;
+  }
+  gs.sync();
+  *mn = lo;
+  *mx = hi;
+}
+
+// Returns T such that exactly k of the n distinct keys key_at(e), e in [0, n), satisfy
+// key >= T (0 < k < n). Radix select with digits of up to 11 bits starting at the highest
+// bit where the smallest and largest key differ: the bits above it are common to every key,
+// so the first histogram spreads over all bins instead of the few bins that keys of similar
+// magnitude share (which would also serialise the shared-memory atomics).
 template <int NT, class KeyAt>
 __device__ uint64_t group_kth_threshold(KeyAt key_at, uint32_t n, uint32_t k, uint32_t rank,
-                                        uint32_t* hist, uint32_t* scratch,
+                                        uint32_t* hist, GroupScratch<NT>& sc,
                                         const GroupSync<NT>& gs) {
   constexpr int BPT = kHistBins / NT;  // bins owned per thread
-  uint64_t prefix = 0, mask = 0;
+  uint64_t mn, mx;
+  group_minmax<NT>(key_at, n, rank, sc, gs, &mn, &mx);
+  int hb = 63 - __clzll(static_cast<long long>(mn ^ mx));
+  uint64_t mask = (hb >= 63) ? 0ull : ~((2ull << hb) - 1ull);
+  uint64_t prefix = mx & mask;
   uint32_t need = k;
 #pragma unroll 1
-  for (int pass = 0; pass < 6; ++pass) {
-    const int shift = radix_shift(pass);
-    const uint32_t digit_mask = (1u << radix_bits(pass)) - 1u;
+  while (hb >= 0) {
+    const int shift = hb >= 10 ? hb - 10 : 0;
+    const uint32_t digit_mask = (2u << (hb - shift)) - 1u;
     for (uint32_t b = rank; b < kHistBins; b += NT) hist[b] = 0;
     gs.sync();
     for (uint32_t e = rank; e < n; e += NT) {
@@ -109,25 +147,26 @@ __device__ uint64_t group_kth_threshold(KeyAt key_at, uint32_t n, uint32_t k, ui
     uint32_t local = 0;
 #pragma unroll
     for (int i = 0; i < BPT; ++i) local += hist[rank * BPT + i];
-    uint32_t acc = group_suffix_exclusive<NT>(local, rank, scratch, gs, nullptr);
+    uint32_t acc = group_suffix_exclusive<NT>(local, rank, sc.w, gs, nullptr);
 #pragma unroll
     for (int i = BPT - 1; i >= 0; --i) {
       const uint32_t c = hist[rank * BPT + i];
       if (acc < need && acc + c >= need) {
-        scratch[NT / 32] = rank * BPT + i;
-        scratch[NT / 32 + 1] = acc;
+        sc.w[NT / 32] = rank * BPT + i;
+        sc.w[NT / 32 + 1] = acc;
       }
       acc += c;
     }
     gs.sync();
-    const uint32_t bin = scratch[NT / 32];
-    const uint32_t above = scratch[NT / 32 + 1];
+    const uint32_t bin = sc.w[NT / 32];
+    const uint32_t above = sc.w[NT / 32 + 1];
     const uint32_t in_bin = hist[bin];
     gs.sync();
     need -= above;
     prefix |= static_cast<uint64_t>(bin) << shift;
     mask |= static_cast<uint64_t>(digit_mask) << shift;
     if (in_bin == need) break;  // every key of this bin is selected
+    hb = shift - 1;
   }
   return prefix;
 }
@@ -136,13 +175,13 @@ __device__ uint64_t group_kth_threshold(KeyAt key_at, uint32_t n, uint32_t k, ui
 // their number. Each thread walks one contiguous segment.
 template <int NT, class KeyAt, class Out>
 __device__ uint32_t group_compact_ge(KeyAt key_at, uint32_t n, uint64_t T, Out out, uint32_t rank,
-                                     uint32_t* scratch, const GroupSync<NT>& gs) {
+                                     GroupScratch<NT>& sc, const GroupSync<NT>& gs) {
   const uint32_t seg = (n + NT - 1) / NT;
   const uint32_t beg = min(n, rank * seg), end = min(n, beg + seg);
   uint32_t c = 0;
   for (uint32_t e = beg; e < end; ++e) c += (key_at(e) >= T) ? 1u : 0u;
   uint32_t total;
-  uint32_t pos = group_prefix_exclusive<NT>(c, rank, scratch, gs, &total);
+  uint32_t pos = group_prefix_exclusive<NT>(c, rank, sc.w, gs, &total);
   for (uint32_t e = beg; e < end; ++e) {
     const uint64_t key = key_at(e);
     if (key >= T) out(pos++, key);
@@ -150,25 +189,85 @@ __device__ uint32_t group_compact_ge(KeyAt key_at, uint32_t n, uint64_t T, Out o
   return total;
 }
 
-// Sorts s[0..P) (P a power of two) in descending key order.
-template <int NT>
-__device__ void group_bitonic_sort_desc(uint64_t* s, uint32_t P, uint32_t rank,
-                                        const GroupSync<NT>& gs) {
-  for (uint32_t size = 2; size <= P; size <<= 1) {
-    for (uint32_t stride = size >> 1; stride > 0; stride >>= 1) {
-      for (uint32_t e = rank; e < (P >> 1); e += NT) {
-        const uint32_t i = 2 * e - (e & (stride - 1));
-        const uint32_t j = i + stride;
-        const bool desc = (i & size) == 0;
-        const uint64_t a = s[i], b = s[j];
-        if ((a < b) == desc) {
-          s[i] = b;
-          s[j] = a;
+// Sorts the 16 keys of one thread in descending order (bitonic network, fully unrolled).
+__device__ __forceinline__ void sort16_desc(uint64_t (&v)[16]) {
+#pragma unroll
+  for (int size = 2; size <= 16; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const bool desc = (i & size) == 0;
+          const uint64_t a = v[i], b = v[j];
+          const bool swap = desc ? (a < b) : (a > b);
+          v[i] = swap ? b : a;
+          v[j] = swap ? a : b;
         }
       }
-      gs.sync();
     }
   }
+}
+
+// Shared-memory index of element x of a sort buffer: one padding slot after every 16 keys,
+// so that the 16-key runs of consecutive threads fall into different banks.
+__device__ __forceinline__ uint32_t spad(uint32_t x) { return x + (x >> 4); }
+constexpr int sort_buffer_len(int P) { return P + P / 16; }
+
+// Sorts P keys (P a power of two, 16 <= P <= 16 * NT) in descending order. load(e) supplies
+// key e (e < P). Each of the first P/16 threads loads 16 keys with a coalesced stride, sorts
+// them in registers and writes them as one run; runs are then merged pairwise, every thread
+// emitting 16 consecutive outputs found by a merge-path search. a and b hold
+// sort_buffer_len(P) keys each (padded layout, see spad). Returns the buffer holding the result.
+template <int NT, class Load>
+__device__ uint64_t* group_merge_sort_desc(Load load, uint64_t* a, uint64_t* b, uint32_t P,
+                                           uint32_t rank, const GroupSync<NT>& gs) {
+  const uint32_t active = P / 16;
+  if (rank < active) {
+    uint64_t v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = load(i * active + rank);
+    sort16_desc(v);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) a[spad(rank * 16 + i)] = v[i];
+  }
+  gs.sync();
+  uint64_t* src = a;
+  uint64_t* dst = b;
+  for (uint32_t r = 16; r < P; r <<= 1) {
+    if (rank < active) {
+      const uint32_t out0 = rank * 16;
+      const uint32_t base = out0 & ~(2 * r - 1);  // start of this pair of runs
+      const uint32_t o = out0 - base;             // output offset within the pair
+      uint32_t lo = o > r ? o - r : 0, hi = o < r ? o : r;
+      while (lo < hi) {  // number of run-A keys among the first o outputs
+        const uint32_t mid = (lo + hi) >> 1;
+        if (src[spad(base + mid)] > src[spad(base + r + o - mid - 1)]) lo = mid + 1;
+        else hi = mid;
+      }
+      uint32_t ia = lo, ib = o - lo;
+      uint64_t va = src[spad(base + (ia < r ? ia : r - 1))];
+      uint64_t vb = src[spad(base + r + (ib < r ? ib : r - 1))];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const bool take_a = ib >= r || (ia < r && va > vb);
+        dst[spad(out0 + i)] = take_a ? va : vb;
+        if (take_a) {
+          ++ia;
+          va = src[spad(base + (ia < r ? ia : r - 1))];
+        } else {
+          ++ib;
+          vb = src[spad(base + r + (ib < r ? ib : r - 1))];
+        }
+      }
+    }
+    gs.sync();
+    uint64_t* t = src;
+    src = dst;
+    dst = t;
+  }
+  return src;
 }
 
 }  // namespace dsa

@@ -2,38 +2,43 @@
 //   sort_rows_kernel   : orders each row's exact top-k keys (prefill winners) by key
 //                        descending = (score descending, index ascending) and writes
 //                        out_idx / out_score with -1 / -inf padding.
-//   decode_topk_kernel : per request, exact top-k of its n_b stored scores (radix select on
-//                        the 64-bit (score, position) key), then the same ordering.
+//   decode_topk_kernel : per request, exact top-k of its n_b stored scores. The scoring kernel
+//                        has already counted the request's scores in 2048 bins of their
+//                        order-preserving top 11 bits; the bin holding the k-th score bounds
+//                        the candidates, which one pass over the scores collects into shared
+//                        memory. An exact radix select there and a merge sort finish the row.
 #include "common.cuh"
 #include "internal.h"
 #include "select.cuh"
 
 namespace dsa {
 
-__device__ __forceinline__ uint32_t next_pow2(uint32_t x) {
-  uint32_t p = 1;
-  while (p < x) p <<= 1;
+__device__ __forceinline__ uint32_t sort_size(uint32_t k) {
+  uint32_t p = 16;
+  while (p < k) p <<= 1;
   return p;
 }
 
-constexpr int kSortThreads = 256;
+constexpr int kSortThreads = 128;
+constexpr int kSortBuf = sort_buffer_len(DSA_MAX_TOPK);
 
 __global__ void __launch_bounds__(kSortThreads)
     sort_rows_kernel(const uint64_t* __restrict__ win, int topk, int32_t* __restrict__ out_idx,
                      float* __restrict__ out_score) {
-  __shared__ uint64_t s[DSA_MAX_TOPK];
+  __shared__ uint64_t a[kSortBuf];
+  __shared__ uint64_t b[kSortBuf];
   const GroupSync<kSortThreads> gs{0};
   const uint32_t rank = threadIdx.x;
   const size_t row = blockIdx.x;
-  const uint32_t P = next_pow2(static_cast<uint32_t>(topk));
-  const uint64_t* src = win + row * topk;
-  for (uint32_t e = rank; e < P; e += kSortThreads) s[e] = (e < static_cast<uint32_t>(topk)) ? src[e] : 0ull;
-  gs.sync();
-  group_bitonic_sort_desc<kSortThreads>(s, P, rank, gs);
-  for (uint32_t e = rank; e < static_cast<uint32_t>(topk); e += kSortThreads) {
-    const uint64_t key = s[e];
-    out_idx[row * topk + e] = key_index(key);
-    if (out_score) out_score[row * topk + e] = key_score(key);
+  const uint32_t k = static_cast<uint32_t>(topk);
+  const uint32_t P = sort_size(k);
+  const uint64_t* src = win + row * k;
+  const uint64_t* s = group_merge_sort_desc<kSortThreads>(
+      [&](uint32_t e) { return e < k ? __ldcs(src + e) : 0ull; }, a, b, P, rank, gs);
+  for (uint32_t e = rank; e < k; e += kSortThreads) {
+    const uint64_t key = s[spad(e)];
+    out_idx[row * k + e] = key_index(key);
+    if (out_score) out_score[row * k + e] = key_score(key);
   }
 }
 
@@ -44,49 +49,126 @@ dsa_status launch_sort_rows(const uint64_t* win, int rows, int topk, int32_t* ou
 }
 
 constexpr int kDecodeTopkThreads = 1024;
+constexpr uint32_t kDecodeCandCap = 8192;
+
+struct DecodeTopkSmem {
+  uint64_t a[kSortBuf];             // sort buffer
+  uint64_t win[DSA_MAX_TOPK];       // the k winners, contiguous
+  uint64_t cand[kDecodeCandCap];    // candidates; later the second sort buffer
+  uint32_t hist[kHistBins];
+  GroupScratch<kDecodeTopkThreads> sc;
+  uint32_t n_cand;
+};
+static_assert(kDecodeCandCap >= static_cast<uint32_t>(kSortBuf), "second sort buffer");
 
 __global__ void __launch_bounds__(kDecodeTopkThreads)
     decode_topk_kernel(const float* __restrict__ scores, int max_len,
-                       const int32_t* __restrict__ seq_lens, int topk,
-                       int32_t* __restrict__ out_idx, float* __restrict__ out_score,
+                       const int32_t* __restrict__ seq_lens, const uint32_t* __restrict__ bins,
+                       int topk, int32_t* __restrict__ out_idx, float* __restrict__ out_score,
                        WsHeader* hdr) {
-  __shared__ uint64_t s[DSA_MAX_TOPK];
-  __shared__ uint32_t hist[kHistBins];
-  __shared__ uint32_t scr[kDecodeTopkThreads / 32 + 2];
+  extern __shared__ uint8_t smem_raw[];
+  DecodeTopkSmem& sm = *reinterpret_cast<DecodeTopkSmem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 15) & ~static_cast<uintptr_t>(15));
   const GroupSync<kDecodeTopkThreads> gs{0};
-  const uint32_t rank = threadIdx.x;
-  const int b = blockIdx.x;
-  int n = seq_lens[b];
+  const uint32_t rank = threadIdx.x, lane = rank & 31u;
+  const int req = blockIdx.x;
+  int n = seq_lens[req];
   if (n < 1 || n > max_len) {
     if (rank == 0) record_error(hdr, DSA_ERR_DEVICE, DETAIL_BAD_SEQ_LEN);
     n = n < 1 ? 1 : max_len;
   }
-  const float* row = scores + static_cast<size_t>(b) * max_len;
-  auto key_at = [&](uint32_t e) { return make_key(row[e], e); };
-  const uint32_t P = next_pow2(static_cast<uint32_t>(topk));
-  const uint32_t un = static_cast<uint32_t>(n), uk = static_cast<uint32_t>(topk);
-  if (un <= uk) {
-    for (uint32_t e = rank; e < P; e += kDecodeTopkThreads) s[e] = (e < un) ? key_at(e) : 0ull;
+  const float* row = scores + static_cast<size_t>(req) * max_len;
+  auto key_at = [&](uint32_t e) { return make_key(__ldcg(row + e), e); };
+  const uint32_t un = static_cast<uint32_t>(n), k = static_cast<uint32_t>(topk);
+  const uint32_t P = sort_size(k);
+  uint32_t n_win = un < k ? un : k;
+
+  if (un > k) {
+    // Boundary bin: the highest bin where the count of scores at or above it reaches k.
+    for (uint32_t b = rank; b < kHistBins; b += kDecodeTopkThreads)
+      sm.hist[b] = bins[static_cast<size_t>(req) * kHistBins + b];
+    if (rank == 0) sm.n_cand = 0;
+    gs.sync();
+    constexpr int BPT = kHistBins / kDecodeTopkThreads;
+    uint32_t local = 0;
+#pragma unroll
+    for (int i = 0; i < BPT; ++i) local += sm.hist[rank * BPT + i];
+    uint32_t acc = group_suffix_exclusive<kDecodeTopkThreads>(local, rank, sm.sc.w, gs, nullptr);
+#pragma unroll
+    for (int i = BPT - 1; i >= 0; --i) {
+      const uint32_t c = sm.hist[rank * BPT + i];
+      if (acc < k && acc + c >= k) {
+        sm.sc.w[kDecodeTopkThreads / 32] = rank * BPT + i;
+        sm.sc.w[kDecodeTopkThreads / 32 + 1] = acc + c;
+      }
+      acc += c;
+    }
+    gs.sync();
+    const uint32_t bstar = sm.sc.w[kDecodeTopkThreads / 32];
+    const uint32_t n_cand = sm.sc.w[kDecodeTopkThreads / 32 + 1];
+    gs.sync();
+    uint64_t T;
+    if (n_cand <= kDecodeCandCap) {
+      // One pass: keys whose bin is at or above the boundary bin, eight loads in flight.
+      for (uint32_t e0 = 0; e0 < un; e0 += 8 * kDecodeTopkThreads) {
+        uint64_t v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t e = e0 + i * kDecodeTopkThreads + rank;
+          v[i] = e < un ? key_at(e) : 0ull;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const bool take = v[i] != 0ull && static_cast<uint32_t>(v[i] >> 53) >= bstar;
+          const uint32_t m = __ballot_sync(0xFFFFFFFFu, take);
+          if (m) {
+            uint32_t base = 0;
+            if (lane == 0) base = atomicAdd(&sm.n_cand, static_cast<uint32_t>(__popc(m)));
+            base = __shfl_sync(0xFFFFFFFFu, base, 0);
+            const uint32_t pos = base + __popc(m & ((1u << lane) - 1u));
+            if (take && pos < kDecodeCandCap) sm.cand[pos] = v[i];
+          }
+        }
+      }
+      gs.sync();
+      const uint32_t got = sm.n_cand < kDecodeCandCap ? sm.n_cand : kDecodeCandCap;
+      if (got != n_cand && rank == 0) record_error(hdr, DSA_ERR_DEVICE, DETAIL_HIST_MISMATCH);
+      auto cand_at = [&](uint32_t e) { return sm.cand[e]; };
+      T = got > k ? group_kth_threshold<kDecodeTopkThreads>(cand_at, got, k, rank, sm.hist, sm.sc, gs)
+                  : 0ull;
+      n_win = group_compact_ge<kDecodeTopkThreads>(
+          cand_at, got, T, [&](uint32_t pos, uint64_t key) { if (pos < k) sm.win[pos] = key; }, rank,
+          sm.sc, gs);
+    } else {
+      // Too many keys share the boundary bin (heavy ties): radix select over global memory.
+      T = group_kth_threshold<kDecodeTopkThreads>(key_at, un, k, rank, sm.hist, sm.sc, gs);
+      n_win = group_compact_ge<kDecodeTopkThreads>(
+          key_at, un, T, [&](uint32_t pos, uint64_t key) { if (pos < k) sm.win[pos] = key; }, rank,
+          sm.sc, gs);
+    }
+    n_win = n_win < k ? n_win : k;
   } else {
-    for (uint32_t e = uk + rank; e < P; e += kDecodeTopkThreads) s[e] = 0ull;
-    const uint64_t T = group_kth_threshold<kDecodeTopkThreads>(key_at, un, uk, rank, hist, scr, gs);
-    group_compact_ge<kDecodeTopkThreads>(key_at, un, T, [&](uint32_t pos, uint64_t key) { if (pos < uk) s[pos] = key; },
-                                         rank, scr, gs);
+    for (uint32_t e = rank; e < un; e += kDecodeTopkThreads) sm.win[e] = key_at(e);
   }
   gs.sync();
-  group_bitonic_sort_desc<kDecodeTopkThreads>(s, P, rank, gs);
-  for (uint32_t e = rank; e < uk; e += kDecodeTopkThreads) {
-    const uint64_t key = s[e];
-    out_idx[static_cast<size_t>(b) * topk + e] = key_index(key);
-    if (out_score) out_score[static_cast<size_t>(b) * topk + e] = key_score(key);
+  const uint64_t* s = group_merge_sort_desc<kDecodeTopkThreads>(
+      [&](uint32_t e) { return e < n_win ? sm.win[e] : 0ull; }, sm.a, sm.cand, P, rank, gs);
+  for (uint32_t e = rank; e < k; e += kDecodeTopkThreads) {
+    const uint64_t key = s[spad(e)];
+    out_idx[static_cast<size_t>(req) * topk + e] = key_index(key);
+    if (out_score) out_score[static_cast<size_t>(req) * topk + e] = key_score(key);
   }
 }
 
-dsa_status launch_decode_topk(const float* scores, int max_len, const int32_t* seq_lens, int B,
-                              int topk, int32_t* out_idx, float* out_score, void* ws,
-                              cudaStream_t stream) {
-  decode_topk_kernel<<<B, kDecodeTopkThreads, 0, stream>>>(
-      scores, max_len, seq_lens, topk, out_idx, out_score, static_cast<WsHeader*>(ws));
+dsa_status launch_decode_topk(const float* scores, int max_len, const int32_t* seq_lens,
+                              const uint32_t* bins, int B, int topk, int32_t* out_idx,
+                              float* out_score, void* ws, cudaStream_t stream) {
+  const size_t smem = sizeof(DecodeTopkSmem) + 16;
+  if (cudaFuncSetAttribute(decode_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  decode_topk_kernel<<<B, kDecodeTopkThreads, smem, stream>>>(
+      scores, max_len, seq_lens, bins, topk, out_idx, out_score, static_cast<WsHeader*>(ws));
   return cuda_status(cudaGetLastError());
 }
 

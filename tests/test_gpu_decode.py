@@ -83,3 +83,36 @@ def test_bad_block_table_is_reported():
     B.dsa_indexer_decode(layer.q, layer.q_scale, layer.w, layer.k_cache, layer.k_scale_cache,
                          table.cuda(), seq.cuda(), 64, workspace=ws)
     assert B.dsa_read_device_status(ws) == (0, 0)
+
+
+def test_decode_heavy_ties_fall_back_to_exact_select():
+    """20000 identical keys in one request (every score equal, so the boundary histogram bin
+    holds more candidates than fit in shared memory) plus a short second request: still exact,
+    ties to the lowest positions."""
+    lens = [20000, 300]
+    nb = [(n + 63) // 64 for n in lens]
+    nblk = sum(nb)
+    key = np.zeros(128, dtype=np.float32)
+    key[:4] = [1.0, 2.0, -1.0, 3.0]
+    kc = np.tile(torch.from_numpy(key).to(torch.float8_e4m3fn).view(torch.uint8).numpy(), (nblk, 64, 1))
+    ks = np.ones((nblk, 64), dtype=np.float32)
+    table = np.full((2, max(nb)), -1, dtype=np.int32)
+    table[0, :nb[0]] = np.arange(nb[0])
+    table[1, :nb[1]] = np.arange(nb[0], nblk)
+    q = np.zeros((2, 64, 128), dtype=np.float32)
+    q[:, :, 0] = 1.0
+    layer = {"q": torch.from_numpy(q).to(torch.float8_e4m3fn).view(torch.uint8).numpy(),
+             "q_scale": np.ones(2, dtype=np.float32), "w": np.full((2, 64), 0.5, dtype=np.float32),
+             "k_cache": kc, "k_scale_cache": ks}
+    seq = np.array(lens, dtype=np.int32)
+    t = {k: torch.from_numpy(np.ascontiguousarray(v)).cuda() for k, v in layer.items()}
+    ws = torch.zeros(B.dsa_decode_workspace_bytes(2, table.shape[1] * 64, 64, 128, 2048),
+                     dtype=torch.uint8, device="cuda")
+    idx, sc = B.dsa_indexer_decode(t["q"], t["q_scale"], t["w"], t["k_cache"], t["k_scale_cache"],
+                                   torch.from_numpy(table).cuda(), torch.from_numpy(seq).cuda(), 2048,
+                                   workspace=ws)
+    torch.cuda.synchronize()
+    ref = O.decode_rows(layer, table, seq, 2048)
+    for b, r in enumerate(ref):
+        check_row(idx[b].cpu().numpy(), sc[b].cpu().numpy(), r, 2048, exact=True)
+    assert B.dsa_read_device_status(ws) == (0, 0)

@@ -134,3 +134,21 @@ def test_overlap_bad_index_is_reported():
     ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
     B.topk_overlap([T, T], 5, workspace=ws)
     assert B.dsa_read_device_status(ws) == (B.DSA_ERR_DEVICE, 18)
+
+
+def test_overlap_wide_index_range_uses_probe_path():
+    """n_keys = 300000 with 9 layers: the per-layer bitmaps no longer fit in shared memory
+    together and the kernel probes one bitmap at a time; counts stay bit-exact."""
+    N, R, topk, n_keys = 8, 40, 512, 300000
+    rng = np.random.default_rng(17)
+    first = np.stack([rng.choice(n_keys, size=topk, replace=False) for _ in range(R)]).astype(np.int32)
+    layers = []
+    for i in range(N):
+        drop = rng.random(first.shape) < 0.2 * i / N   # layer i keeps ~(1 - 0.2 i/N) of layer 0
+        layers.append(np.where(drop, -1, first).astype(np.int32))
+    layers.append(np.concatenate([first[:, : topk // 2], np.full((R, topk - topk // 2), -1, np.int32)], 1))
+    counts, valid, overlap = B.topk_overlap([torch.from_numpy(T).cuda() for T in layers], n_keys)
+    torch.cuda.synchronize()
+    ref_c, ref_v, ref_o = O.topk_overlap(layers)
+    assert counts.cpu().numpy().astype(np.uint64).tolist() == ref_c.tolist()
+    assert int(valid.item()) == ref_v
