@@ -91,6 +91,20 @@ __device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t count, bool 
   return out != 0;
 }
 
+// Named barrier that also ORs a predicate across the participating threads.
+__device__ __forceinline__ bool named_bar_or(uint32_t id, uint32_t count, bool pred) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %3, 0;\n\t"
+      "bar.red.or.pred po, %1, %2, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(out)
+      : "r"(id), "r"(count), "r"(pred ? 1u : 0u)
+      : "memory");
+  return out != 0;
+}
+
 // Order-preserving map of an fp32 score to uint32 (larger score -> larger key).
 __device__ __forceinline__ uint32_t float_to_ordered(float f) {
   uint32_t u = __float_as_uint(f);

@@ -46,20 +46,24 @@ struct DecodeLaunch {
   int num_sms;
 };
 
-// Candidate-buffer capacity (entries) per query of the streaming prefill top-k.
-inline uint32_t prefill_cand_cap(int topk) {
-  uint32_t c = 2u * static_cast<uint32_t>(topk) + 256u;
-  return (c + 127u) & ~127u;
+// Candidate-buffer capacity (entries) per query of the streaming prefill top-k: four warp
+// segments of cap/4 entries. A segment is cut back as soon as it holds more than cap/4 - 32
+// keys (a tile adds at most 32), and a cut-back leaves at most (k + 131) / 4 keys in it.
+__host__ __device__ constexpr uint32_t prefill_cand_cap(int topk) {
+  return (2u * static_cast<uint32_t>(topk) + 512u + 127u) & ~127u;
 }
+constexpr uint32_t kPrefillCapMax = prefill_cand_cap(DSA_MAX_TOPK);
 inline int prefill_queries_per_block(int H) { return 2 * (256 / H); }
 
 size_t prefill_workspace_bytes(int Lq, int H, int d, int topk, int num_sms);
 size_t decode_workspace_bytes(int B, int max_len, int H, int d, int topk);
 
 dsa_status launch_prefill(const PrefillLaunch& a);
+// Exact top-k of every row's candidate buffer, ordered and written to out_idx / out_score.
+dsa_status launch_prefill_finish(const uint64_t* cand, const uint32_t* counts, uint32_t cap,
+                                 int rows, int topk, int32_t* out_idx, float* out_score,
+                                 cudaStream_t stream);
 dsa_status launch_decode(const DecodeLaunch& a);
-dsa_status launch_sort_rows(const uint64_t* win, int rows, int topk, int32_t* out_idx,
-                            float* out_score, cudaStream_t stream);
 dsa_status launch_decode_topk(const float* scores, int max_len, const int32_t* seq_lens,
                               const uint32_t* bins, int B, int topk, int32_t* out_idx,
                               float* out_score, void* ws, cudaStream_t stream);

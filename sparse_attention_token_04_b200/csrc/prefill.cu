@@ -1,26 +1,30 @@
-// Fused prefill lightning indexer for sm_100a.
+// Fused prefill lightning indexer for sm_100a: scores every causal (query, key) pair on the
+// tensor cores and streams, per query, the keys that can still enter its top-k into that
+// query's candidate buffer in the workspace. prefill_finish_kernel (topk.cu) then takes the
+// exact top-k of each buffer. The L x L score matrix is never stored.
 //
-// One persistent CTA per SM walks query blocks (heaviest first, snake order over CTAs).
-// For a block of QB queries it streams the causal key range in tiles of 128 keys:
+// One persistent CTA per SM walks query blocks (heaviest first, snake order over CTAs). For a
+// block of QB queries it streams the causal key range in tiles of 128 keys:
 //   warp 0      TMA producer: the block's Q rows (two 256-row B operands) once, then one
 //               [128 keys x d] FP8 K tile per pipeline stage;
 //   warp 1      one thread issues tcgen05.mma kind::f8f6f4 (M = 128 keys, N = 256 =
 //               (256/H) queries x H heads, K = d), FP32 accumulators in TMEM, two
 //               256-column accumulators so the epilogue of one overlaps the MMA of the other;
 //   warps 4-11  two epilogue warpgroups, one per accumulator. Thread = key (its TMEM lane):
-//               it reads the key's H head dot products of each query, applies
-//               ReLU, the head weights, then the query and key scales, masks s > t, and
-//               streams keys that can still enter the top-k into a per-query candidate
-//               buffer (workspace). A nearly full buffer is staged in shared memory and cut
-//               back to exactly topk keys by an exact radix select, which also raises the
-//               query's insertion threshold.
-// After the last tile every query's buffer is reduced to exactly its top-k keys and written
-// to the winners array; the row sort (topk.cu) orders them. The L x L score matrix is never
-// stored.
+//               it reads the key's H head dot products of each query, applies ReLU, the head
+//               weights, then the query and key scales, masks s > t, and appends the keys at
+//               or above the query's threshold to its warp's segment of the query's buffer
+//               (no atomics: the segment's count lives in a register of the warp).
+// When a segment may overflow on the next tile, the warpgroup cuts that query's buffer back to
+// the keys at or above the histogram bin holding its k-th key (k to k + 128 keys), spread
+// evenly over the four segments, and raises the query's threshold to that bin's lower edge.
+// A key below the threshold has k buffered keys above it, so dropping it is exact.
 //
 // ReLU on the FMA pipe: D = q8.k8 with |D| <= d * 448^2 < 2^25, so
 // max(D, 0) = 2^25 * sat(D * 2^-25) exactly (power-of-two scalings, no clipping at 1), and
 // the 2^25 is folded into the stored head weights.
+#include <cstddef>
+
 #include "common.cuh"
 #include "internal.h"
 #include "select.cuh"
@@ -37,13 +41,17 @@ struct PCfg {
   static constexpr int KTILE = BN * D;      // bytes of one A operand
   static constexpr int KSTEPS = D / 32;     // K = 32 per FP8 MMA instruction
   static constexpr int THREADS = 384;
-  static constexpr int NP = (H >= 32) ? 4 : 1;  // partial sums per query (ILP)
   static constexpr uint32_t IDESC = make_idesc_f8(128, 256);
   static_assert(D == 64 || D == 128, "d");
   static_assert(H == 8 || H == 64, "H");
 };
 
-constexpr int kCandCapMax = 2 * DSA_MAX_TOPK + 256;
+// Selection state of one epilogue warpgroup's cut-backs.
+struct __align__(16) CutState {
+  uint32_t hist[kHistBins];         // zero between cut-backs
+  GroupScratch<128> sc;
+  uint64_t stage[kPrefillCapMax];   // the buffer being cut, contiguous
+};
 
 template <int H, int D>
 struct PSmem {
@@ -53,10 +61,9 @@ struct PSmem {
   float wq[C::QB][H];
   float sq[C::QB];
   uint64_t thr[C::QB];
-  uint32_t cnt[C::QB];
-  uint32_t hist[2][kHistBins];
-  GroupScratch<128> gsc[2];
-  uint64_t stage[2][kCandCapMax];   // a candidate buffer staged for a cut-back
+  uint32_t wcnt[C::QB][4];  // per query: keys in each warp's segment, exchanged at cut-backs
+  uint32_t cflag[2];        // per warpgroup: queries whose buffer needs a cut-back
+  CutState cut[2];
   uint64_t kfull[C::STAGES];
   uint64_t kempty[C::STAGES];
   uint64_t qfull, qempty, accfull[2], accempty[2], drain;
@@ -64,20 +71,12 @@ struct PSmem {
   int abort;
 };
 
-// Copies n candidate keys from global memory into shared memory, eight independent loads in
-// flight per thread.
-__device__ __forceinline__ void stage_keys(const uint64_t* __restrict__ src, uint32_t n,
-                                           uint64_t* __restrict__ dst, uint32_t rank) {
-  uint32_t e = rank;
-  for (; e + 7 * 128 < n; e += 8 * 128) {
-    uint64_t v[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = __ldcg(src + e + i * 128);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) dst[e + i * 128] = v[i];
-  }
-  for (; e < n; e += 128) dst[e] = __ldcg(src + e);
-}
+using PSmemH64 = PSmem<64, 128>;
+using PSmemH8 = PSmem<8, 64>;
+static_assert(sizeof(PSmemH64) + 1024 <= 232448, "shared memory of the H=64 kernel");
+static_assert(sizeof(PSmemH8) + 1024 <= 232448, "shared memory of the H=8 kernel");
+static_assert(offsetof(PSmemH64, wq) % 16 == 0 && offsetof(PSmemH8, wq) % 16 == 0,
+              "vectorised weight access");
 
 struct PrefillParams {
   const float* q_scale;
@@ -85,12 +84,58 @@ struct PrefillParams {
   const float* k_scale;
   int32_t Lk, q_pos0, Lq, topk;
   int32_t nqb;
-  uint32_t cap;
-  uint64_t* cand;
-  uint64_t* win;
+  uint32_t cap;        // candidate entries per row: four segments of cap / 4
+  uint64_t* cand;      // [Lq][cap]
+  uint32_t* counts;    // [Lq][4] keys in each segment after the scan
   WsHeader* hdr;
   uint64_t budget_ns;
 };
+
+// Cut-back of one query's candidate buffer by its warpgroup (128 threads on named barrier
+// bar_id). The four segment counts are in wcnt[0..3]. Stages the segments contiguously in
+// shared memory; with more than k + 128 keys it finds the lower edge T of the histogram bin
+// holding the k-th key (k <= count(keys >= T) <= k + 128) and keeps the keys >= T, otherwise it
+// keeps every key. The kept keys are written back dealt round-robin over the four segments;
+// wcnt and (after a select) *thr are updated. One out-of-line copy serves every call site.
+__device__ __noinline__ void cut_back(uint64_t* buf, uint32_t segcap, uint32_t* wcnt,
+                                      uint64_t* thr, CutState* cs, uint32_t k, uint32_t rank,
+                                      uint32_t bar_id) {
+  const GroupSync<128> gs{bar_id};
+  const uint32_t lane = rank & 31u, w = rank >> 5;
+  uint32_t n = 0, off = 0;
+  for (uint32_t i = 0; i < 4; ++i) {
+    const uint32_t c = wcnt[i];
+    off += (i < w) ? c : 0u;
+    n += c;
+  }
+  const uint32_t c = wcnt[w];
+  const uint64_t* src = buf + w * segcap;
+  uint64_t* st = cs->stage;
+  uint32_t e = lane;
+  for (; e + 96 < c; e += 128) {
+    const uint64_t a0 = __ldcg(src + e), a1 = __ldcg(src + e + 32), a2 = __ldcg(src + e + 64),
+                   a3 = __ldcg(src + e + 96);
+    st[off + e] = a0;
+    st[off + e + 32] = a1;
+    st[off + e + 64] = a2;
+    st[off + e + 96] = a3;
+  }
+  for (; e < c; e += 32) st[off + e] = __ldcg(src + e);
+  gs.sync();
+  auto key_at = [st](uint32_t i) { return st[i]; };
+  uint64_t T = 0;
+  if (n > k + 128u) {
+    uint32_t cnt;
+    T = group_select_threshold<128>(key_at, n, k, k + 128u, rank, cs->hist, cs->sc, gs, &cnt);
+  }
+  const uint32_t kept = group_compact_ge<128>(
+      key_at, n, T,
+      [buf, segcap](uint32_t pos, uint64_t key) { buf[(pos & 3u) * segcap + (pos >> 2)] = key; },
+      rank, cs->sc, gs);
+  if (rank < 4) wcnt[rank] = (kept + 3u - rank) >> 2;
+  if (rank == 0 && T != 0) *thr = T;
+  gs.sync();
+}
 
 template <int H, int D>
 __global__ void __launch_bounds__(384, 1)
@@ -136,9 +181,6 @@ __global__ void __launch_bounds__(384, 1)
   auto ntiles_of = [&](int qb) -> int {
     const int last_row = min(qb * C::QB + C::QB, p.Lq) - 1;
     return (p.q_pos0 + last_row) / C::BN + 1;
-  };
-  auto cand_buf = [&](int qidx) -> uint64_t* {
-    return p.cand + (static_cast<size_t>(cta) * C::QB + qidx) * p.cap;
   };
 
   if (warp == 0) {
@@ -228,15 +270,19 @@ __global__ void __launch_bounds__(384, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------------ epilogue
-    const uint32_t g = (warp - 4) >> 2;       // accumulator / warpgroup
-    const uint32_t wl = warp & 3u;            // TMEM lane quarter of this warp
+    const uint32_t g = (warp - 4) >> 2;   // accumulator / warpgroup
+    const uint32_t wl = warp & 3u;        // TMEM lane quarter = buffer segment of this warp
     const uint32_t rank = threadIdx.x - 128u * (1u + g);
     const GroupSync<128> gs{1u + g};
-    uint32_t* hist = sm.hist[g];
-    GroupScratch<128>& scr = sm.gsc[g];
-    uint64_t* stage = sm.stage[g];
+    CutState* cs = &sm.cut[g];
     const uint32_t taddr0 = tmem + g * 256 + ((wl * 32u) << 16);
     const int qbase = static_cast<int>(g) * C::QPM;
+    const uint32_t k = static_cast<uint32_t>(p.topk);
+    const uint32_t segcap = p.cap / 4u;
+    const uint32_t trigger = segcap - 32u;  // above it the next tile could overflow the segment
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int i = rank; i < kHistBins; i += 128) cs->hist[i] = 0u;  // the selects keep it zero
+    if (rank == 0) sm.cflag[g] = 0u;
     uint32_t use = 0;
     bool ok = true;
     for (int r = 0; ok; ++r) {
@@ -252,108 +298,129 @@ __global__ void __launch_bounds__(384, 1)
         const int row = row_base + qi;
         sm.sq[qbase + qi] = (row < p.Lq) ? __ldg(&p.q_scale[row]) : 0.0f;
         sm.thr[qbase + qi] = 0;
-        sm.cnt[qbase + qi] = 0;
       }
       gs.sync();
+      uint32_t cw[C::QPM];  // keys in this warp's segment, per query (warp-uniform)
+#pragma unroll
+      for (int qi = 0; qi < C::QPM; ++qi) cw[qi] = 0u;
       const int nt = ntiles_of(qb);
-      for (int tile = 0; tile < nt; ++tile) {
-        const int s = tile * C::BN + static_cast<int>(wl * 32u + lane);
-        const float sk = (s < p.Lk) ? __ldg(&p.k_scale[s]) : 0.0f;
+      int s = static_cast<int>(wl * 32u + lane);
+      float sk_next = (s < p.Lk) ? __ldg(&p.k_scale[s]) : 0.0f;
+      bool good = true;
+      for (int tile = 0; tile < nt; ++tile, s += C::BN) {
+        const float sk = sk_next;
+        sk_next = (s + C::BN < p.Lk) ? __ldg(&p.k_scale[s + C::BN]) : 0.0f;
         const bool got = mbar_wait(&sm.accfull[g], use & 1u, ctl, DETAIL_WAIT_ACCFULL);
+        good = good && got;
         __syncwarp();
         tc_fence_after();
-        float part[C::QPM][C::NP];
-#pragma unroll
-        for (int qi = 0; qi < C::QPM; ++qi)
-#pragma unroll
-          for (int pp = 0; pp < C::NP; ++pp) part[qi][pp] = 0.0f;
+        float score_part[C::QPM];
         uint32_t ra[32], rb[32];
         tmem_ld_32x32b_x32(taddr0, ra);
         tmem_wait_ld_regs(ra);
+        if constexpr (H == 64) {
+          // 4 queries x 64 heads: packed FMA over head pairs, four float2 partial sums per query.
+          float2 acc[C::QPM][4];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint32_t(&cur)[32] = (c & 1) ? rb : ra;
-          uint32_t(&nxt)[32] = (c & 1) ? ra : rb;
-          if (c + 1 < 8) tmem_ld_32x32b_x32(taddr0 + (c + 1) * 32, nxt);
+          for (int qi = 0; qi < C::QPM; ++qi)
 #pragma unroll
-          for (int j = 0; j < 32; j += 4) {
-            const int col = c * 32 + j;
-            const int qi = col / H, h = col % H;
-            const float4 wv = *reinterpret_cast<const float4*>(&sm.wq[qbase + qi][h]);
-            part[qi][(j + 0) % C::NP] = fmaf(wv.x, __saturatef(__uint_as_float(cur[j + 0]) * 0x1p-25f), part[qi][(j + 0) % C::NP]);
-            part[qi][(j + 1) % C::NP] = fmaf(wv.y, __saturatef(__uint_as_float(cur[j + 1]) * 0x1p-25f), part[qi][(j + 1) % C::NP]);
-            part[qi][(j + 2) % C::NP] = fmaf(wv.z, __saturatef(__uint_as_float(cur[j + 2]) * 0x1p-25f), part[qi][(j + 2) % C::NP]);
-            part[qi][(j + 3) % C::NP] = fmaf(wv.w, __saturatef(__uint_as_float(cur[j + 3]) * 0x1p-25f), part[qi][(j + 3) % C::NP]);
+            for (int a = 0; a < 4; ++a) acc[qi][a] = make_float2(0.0f, 0.0f);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint32_t(&cur)[32] = (c & 1) ? rb : ra;
+            uint32_t(&nxt)[32] = (c & 1) ? ra : rb;
+            if (c + 1 < 8) tmem_ld_32x32b_x32(taddr0 + (c + 1) * 32, nxt);
+            const int qi = c >> 1;
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              const int h = (c & 1) * 32 + j;
+              const float4 wv = *reinterpret_cast<const float4*>(&sm.wq[qbase + qi][h]);
+              const float r0 = __saturatef(__uint_as_float(cur[j + 0]) * 0x1p-25f);
+              const float r1 = __saturatef(__uint_as_float(cur[j + 1]) * 0x1p-25f);
+              const float r2 = __saturatef(__uint_as_float(cur[j + 2]) * 0x1p-25f);
+              const float r3 = __saturatef(__uint_as_float(cur[j + 3]) * 0x1p-25f);
+              const int a = ((j >> 2) & 1) * 2;
+              acc[qi][a] = __ffma2_rn(make_float2(wv.x, wv.y), make_float2(r0, r1), acc[qi][a]);
+              acc[qi][a + 1] = __ffma2_rn(make_float2(wv.z, wv.w), make_float2(r2, r3), acc[qi][a + 1]);
+            }
+            if (c + 1 < 8) tmem_wait_ld_regs(nxt);
           }
-          if (c + 1 < 8) tmem_wait_ld_regs(nxt);
+#pragma unroll
+          for (int qi = 0; qi < C::QPM; ++qi)
+            score_part[qi] = ((acc[qi][0].x + acc[qi][0].y) + (acc[qi][1].x + acc[qi][1].y)) +
+                             ((acc[qi][2].x + acc[qi][2].y) + (acc[qi][3].x + acc[qi][3].y));
+        } else {
+          // 32 queries x 8 heads: one scalar chain per query, four queries per chunk.
+#pragma unroll
+          for (int qi = 0; qi < C::QPM; ++qi) score_part[qi] = 0.0f;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint32_t(&cur)[32] = (c & 1) ? rb : ra;
+            uint32_t(&nxt)[32] = (c & 1) ? ra : rb;
+            if (c + 1 < 8) tmem_ld_32x32b_x32(taddr0 + (c + 1) * 32, nxt);
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              const int col = c * 32 + j;
+              const int qi = col / H, h = col % H;
+              const float4 wv = *reinterpret_cast<const float4*>(&sm.wq[qbase + qi][h]);
+              score_part[qi] = fmaf(wv.x, __saturatef(__uint_as_float(cur[j + 0]) * 0x1p-25f), score_part[qi]);
+              score_part[qi] = fmaf(wv.y, __saturatef(__uint_as_float(cur[j + 1]) * 0x1p-25f), score_part[qi]);
+              score_part[qi] = fmaf(wv.z, __saturatef(__uint_as_float(cur[j + 2]) * 0x1p-25f), score_part[qi]);
+              score_part[qi] = fmaf(wv.w, __saturatef(__uint_as_float(cur[j + 3]) * 0x1p-25f), score_part[qi]);
+            }
+            if (c + 1 < 8) tmem_wait_ld_regs(nxt);
+          }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.accempty[g]);
         ++use;
 
+        // Inserts into this warp's own segment: no atomics, the count lives in a register.
+        uint32_t flags = 0u;
 #pragma unroll
         for (int qi = 0; qi < C::QPM; ++qi) {
-          float acc = part[qi][0];
-#pragma unroll
-          for (int pp = 1; pp < C::NP; ++pp) acc += part[qi][pp];
           const int row = row_base + qi;
           const bool valid = (row < p.Lq) && (s <= p.q_pos0 + row);
-          const float score = (acc * sm.sq[qbase + qi]) * sk;
+          const float score = (score_part[qi] * sm.sq[qbase + qi]) * sk;
           const uint64_t key = make_key(score, static_cast<uint32_t>(s));
           const bool take = valid && key >= sm.thr[qbase + qi];
           const uint32_t m = __ballot_sync(0xFFFFFFFFu, take);
-          if (m) {
-            uint32_t base = 0;
-            if (lane == 0) base = atomicAdd(&sm.cnt[qbase + qi], static_cast<uint32_t>(__popc(m)));
-            base = __shfl_sync(0xFFFFFFFFu, base, 0);
-            if (take) cand_buf(qbase + qi)[base + __popc(m & ((1u << lane) - 1u))] = key;
-          }
+          const uint32_t pos = cw[qi] + __popc(m & lt);
+          if (take) p.cand[static_cast<size_t>(row) * p.cap + wl * segcap + pos] = key;
+          cw[qi] += __popc(m);
+          flags |= (cw[qi] > trigger) ? (1u << qi) : 0u;
         }
-        ok = named_bar_and(1u + g, 128, ok && got);
-        if (!ok) break;
-        // Cut any nearly full candidate buffer back to exactly topk keys: stage it in shared
-        // memory, find the threshold there, write the survivors back to the buffer's front.
-        for (int qi = 0; qi < C::QPM; ++qi) {
-          const uint32_t n = sm.cnt[qbase + qi];
-          if (n <= p.cap - 128u) continue;
-          uint64_t* buf = cand_buf(qbase + qi);
-          stage_keys(buf, n, stage, rank);
-          gs.sync();
-          auto key_at = [&](uint32_t e) { return stage[e]; };
-          const uint32_t k = static_cast<uint32_t>(p.topk);
-          const uint64_t T = group_kth_threshold<128>(key_at, n, k, rank, hist, scr, gs);
-          group_compact_ge<128>(key_at, n, T,
-                                [&](uint32_t pos, uint64_t key) { if (pos < k) buf[pos] = key; },
-                                rank, scr, gs);
-          if (rank == 0) {
-            sm.thr[qbase + qi] = T;
-            sm.cnt[qbase + qi] = k;
+        // One decision for the whole warpgroup: the barrier ORs the warps' requests, and the
+        // flag word written before it is visible to every warp after it.
+        if (flags && lane == 0) atomicOr(&sm.cflag[g], flags);
+        if (named_bar_or(1u + g, 128, flags != 0u)) {
+          const uint32_t mask = *reinterpret_cast<volatile uint32_t*>(&sm.cflag[g]);
+          if (lane == 0) {
+#pragma unroll
+            for (int qi = 0; qi < C::QPM; ++qi) sm.wcnt[qbase + qi][wl] = cw[qi];
           }
           gs.sync();
+          if (rank == 0) sm.cflag[g] = 0u;
+#pragma unroll 1
+          for (int qi = 0; qi < C::QPM; ++qi) {
+            if ((mask >> qi) & 1u)
+              cut_back(p.cand + static_cast<size_t>(row_base + qi) * p.cap, segcap,
+                       sm.wcnt[qbase + qi], &sm.thr[qbase + qi], cs, k, rank, 1u + g);
+          }
+#pragma unroll
+          for (int qi = 0; qi < C::QPM; ++qi) cw[qi] = sm.wcnt[qbase + qi][wl];
         }
       }
+      ok = named_bar_and(1u + g, 128, ok && good);
       if (!ok) break;
-      // Final top-k of every query of this warpgroup -> winners[row][0..topk).
-      for (int qi = 0; qi < C::QPM; ++qi) {
-        const int row = row_base + qi;
-        if (row >= p.Lq) break;
-        const uint32_t n = sm.cnt[qbase + qi];
-        const uint32_t k = static_cast<uint32_t>(p.topk);
-        const uint64_t* buf = cand_buf(qbase + qi);
-        uint64_t* dst = p.win + static_cast<size_t>(row) * p.topk;
-        if (n > k) {
-          stage_keys(buf, n, stage, rank);
-          gs.sync();
-          auto key_at = [&](uint32_t e) { return stage[e]; };
-          const uint64_t T = group_kth_threshold<128>(key_at, n, k, rank, hist, scr, gs);
-          group_compact_ge<128>(key_at, n, T,
-                                [&](uint32_t pos, uint64_t key) { if (pos < k) dst[pos] = key; },
-                                rank, scr, gs);
-        } else {
-          for (uint32_t e = rank; e < k; e += 128) dst[e] = (e < n) ? buf[e] : 0ull;
+      // The segment counts of every query of this warpgroup, for the finishing kernel.
+      if (lane == 0) {
+#pragma unroll
+        for (int qi = 0; qi < C::QPM; ++qi) {
+          const int row = row_base + qi;
+          if (row < p.Lq) p.counts[static_cast<size_t>(row) * 4 + wl] = cw[qi];
         }
-        gs.sync();
       }
     }
   }
@@ -394,20 +461,22 @@ static dsa_status launch_prefill_t(const PrefillLaunch& a) {
   p.cap = prefill_cand_cap(a.topk);
   p.hdr = reinterpret_cast<WsHeader*>(base);
   p.cand = reinterpret_cast<uint64_t*>(base + DSA_WS_HEADER_BYTES);
-  const size_t cand_bytes = static_cast<size_t>(a.num_sms) * C::QB * p.cap * sizeof(uint64_t);
-  p.win = reinterpret_cast<uint64_t*>(base + DSA_WS_HEADER_BYTES + cand_bytes);
+  p.counts = reinterpret_cast<uint32_t*>(base + DSA_WS_HEADER_BYTES +
+                                         static_cast<size_t>(a.Lq) * p.cap * sizeof(uint64_t));
   p.budget_ns = a.budget_ns;
   kern<<<grid, C::THREADS, smem, a.stream>>>(tq, tk, p);
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
-  return launch_sort_rows(p.win, a.Lq, a.topk, a.out_idx, a.out_score, a.stream);
+  return launch_prefill_finish(p.cand, p.counts, p.cap, a.Lq, a.topk, a.out_idx, a.out_score,
+                               a.stream);
 }
 
 size_t prefill_workspace_bytes(int Lq, int H, int d, int topk, int num_sms) {
+  (void)H;
   (void)d;
-  const size_t qb = static_cast<size_t>(prefill_queries_per_block(H));
-  const size_t cand = static_cast<size_t>(num_sms) * qb * prefill_cand_cap(topk) * sizeof(uint64_t);
-  const size_t win = static_cast<size_t>(Lq) * topk * sizeof(uint64_t);
-  return DSA_WS_HEADER_BYTES + cand + win;
+  (void)num_sms;
+  const size_t cand = static_cast<size_t>(Lq) * prefill_cand_cap(topk) * sizeof(uint64_t);
+  const size_t counts = static_cast<size_t>(Lq) * 4 * sizeof(uint32_t);
+  return DSA_WS_HEADER_BYTES + cand + counts;
 }
 
 dsa_status launch_prefill(const PrefillLaunch& a) {

@@ -16,10 +16,10 @@ struct GroupSync {
   __device__ __forceinline__ void sync() const { named_bar(bar_id, NT); }
 };
 
-// Scratch words a group needs: NT/32 + 2 (u32) and 2 * NT/32 (u64).
+// Scratch words a group needs: NT/32 + 4 (u32) and 2 * NT/32 (u64).
 template <int NT>
 struct GroupScratch {
-  uint32_t w[NT / 32 + 2];
+  uint32_t w[NT / 32 + 4];
   uint64_t w64[2 * (NT / 32)];
 };
 
@@ -116,28 +116,31 @@ __device__ void group_minmax(KeyAt key_at, uint32_t n, uint32_t rank, GroupScrat
   *mx = hi;
 }
 
-// Returns T such that exactly k of the n distinct keys key_at(e), e in [0, n), satisfy
-// key >= T (0 < k < n). Radix select with digits of up to 11 bits starting at the highest
-// bit where the smallest and largest key differ: the bits above it are common to every key,
-// so the first histogram spreads over all bins instead of the few bins that keys of similar
-// magnitude share (which would also serialise the shared-memory atomics).
+// Radix selection on the n distinct keys key_at(e), e in [0, n), with 0 < k < n.
+// Digits of up to 11 bits start at the highest bit where the smallest and largest key differ
+// (the bits above it are common to every key), so the first histogram spreads over all bins
+// instead of the few bins that keys of similar magnitude share. After each pass the highest bin
+// holding the k-th key is known; with `taken` keys in higher bins and `in_bin` keys in it,
+// every key >= the bin's lower edge E is among the taken + in_bin largest. The select stops as
+// soon as taken + in_bin <= relax_limit and returns E: relax_limit = k gives the exact k-th
+// threshold (exactly k keys >= E); a larger limit returns after fewer passes with
+// k <= count(keys >= E) <= relax_limit. *count receives count(keys >= E).
+// `hist` (kHistBins words) must be zero on entry and is zero again on return.
 template <int NT, class KeyAt>
-__device__ uint64_t group_kth_threshold(KeyAt key_at, uint32_t n, uint32_t k, uint32_t rank,
-                                        uint32_t* hist, GroupScratch<NT>& sc,
-                                        const GroupSync<NT>& gs) {
+__device__ uint64_t group_select_threshold(KeyAt key_at, uint32_t n, uint32_t k, uint32_t relax_limit,
+                                           uint32_t rank, uint32_t* hist, GroupScratch<NT>& sc,
+                                           const GroupSync<NT>& gs, uint32_t* count) {
   constexpr int BPT = kHistBins / NT;  // bins owned per thread
   uint64_t mn, mx;
   group_minmax<NT>(key_at, n, rank, sc, gs, &mn, &mx);
   int hb = 63 - __clzll(static_cast<long long>(mn ^ mx));
   uint64_t mask = (hb >= 63) ? 0ull : ~((2ull << hb) - 1ull);
   uint64_t prefix = mx & mask;
-  uint32_t need = k;
+  uint32_t need = k, taken = 0;
 #pragma unroll 1
-  while (hb >= 0) {
+  while (true) {
     const int shift = hb >= 10 ? hb - 10 : 0;
     const uint32_t digit_mask = (2u << (hb - shift)) - 1u;
-    for (uint32_t b = rank; b < kHistBins; b += NT) hist[b] = 0;
-    gs.sync();
     for (uint32_t e = rank; e < n; e += NT) {
       const uint64_t key = key_at(e);
       if ((key & mask) == prefix)
@@ -154,39 +157,155 @@ __device__ uint64_t group_kth_threshold(KeyAt key_at, uint32_t n, uint32_t k, ui
       if (acc < need && acc + c >= need) {
         sc.w[NT / 32] = rank * BPT + i;
         sc.w[NT / 32 + 1] = acc;
+        sc.w[NT / 32 + 2] = c;
       }
       acc += c;
     }
     gs.sync();
     const uint32_t bin = sc.w[NT / 32];
     const uint32_t above = sc.w[NT / 32 + 1];
-    const uint32_t in_bin = hist[bin];
+    const uint32_t in_bin = sc.w[NT / 32 + 2];
+#pragma unroll
+    for (int i = 0; i < BPT; ++i) hist[rank * BPT + i] = 0u;  // ready for the next pass / call
     gs.sync();
     need -= above;
+    taken += above;
     prefix |= static_cast<uint64_t>(bin) << shift;
     mask |= static_cast<uint64_t>(digit_mask) << shift;
-    if (in_bin == need) break;  // every key of this bin is selected
+    if (taken + in_bin <= relax_limit || shift == 0) {
+      *count = taken + in_bin;
+      return prefix;
+    }
     hb = shift - 1;
   }
-  return prefix;
 }
 
-// Stable compaction: writes, in order, the keys key_at(e) >= T to out(pos, key) and returns
-// their number. Each thread walks one contiguous segment.
+// Exact k-th threshold: exactly k keys are >= the returned value.
+template <int NT, class KeyAt>
+__device__ uint64_t group_kth_threshold(KeyAt key_at, uint32_t n, uint32_t k, uint32_t rank,
+                                        uint32_t* hist, GroupScratch<NT>& sc,
+                                        const GroupSync<NT>& gs) {
+  uint32_t cnt;
+  return group_select_threshold<NT>(key_at, n, k, k, rank, hist, sc, gs, &cnt);
+}
+
+// Stable compaction: writes the keys key_at(e) >= T, e in [0, n), in element order to
+// out(pos, key) and returns their number. Warp w owns the elements
+// [w * per, (w + 1) * per); a ballot pass counts its keeps, one barrier exchanges the warps'
+// totals, and a ballot pass writes. No atomics; loads within a pass are independent.
 template <int NT, class KeyAt, class Out>
 __device__ uint32_t group_compact_ge(KeyAt key_at, uint32_t n, uint64_t T, Out out, uint32_t rank,
                                      GroupScratch<NT>& sc, const GroupSync<NT>& gs) {
-  const uint32_t seg = (n + NT - 1) / NT;
-  const uint32_t beg = min(n, rank * seg), end = min(n, beg + seg);
-  uint32_t c = 0;
-  for (uint32_t e = beg; e < end; ++e) c += (key_at(e) >= T) ? 1u : 0u;
-  uint32_t total;
-  uint32_t pos = group_prefix_exclusive<NT>(c, rank, sc.w, gs, &total);
-  for (uint32_t e = beg; e < end; ++e) {
-    const uint64_t key = key_at(e);
-    if (key >= T) out(pos++, key);
+  constexpr int NW = NT / 32;
+  const uint32_t lane = rank & 31u, warp = rank >> 5;
+  const uint32_t per = (((n + NW - 1) / NW) + 31u) & ~31u;
+  const uint32_t beg = min(n, warp * per), end = min(n, beg + per);
+  uint32_t mine = 0;
+  for (uint32_t e0 = beg; e0 < end; e0 += 128) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t e = e0 + i * 32 + lane;
+      mine += __popc(__ballot_sync(0xFFFFFFFFu, e < end && key_at(e) >= T));
+    }
   }
+  if (lane == 0) sc.w[warp] = mine;
+  gs.sync();
+  uint32_t base = 0, total = 0;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) {
+    const uint32_t t = sc.w[w];
+    base += (w < static_cast<int>(warp)) ? t : 0u;
+    total += t;
+  }
+  const uint32_t lt = (1u << lane) - 1u;
+  for (uint32_t e0 = beg; e0 < end; e0 += 32) {
+    const uint32_t e = e0 + lane;
+    const uint64_t key = e < end ? key_at(e) : 0ull;
+    const bool keep = e < end && key >= T;
+    const uint32_t m = __ballot_sync(0xFFFFFFFFu, keep);
+    if (keep) out(base + __popc(m & lt), key);
+    base += __popc(m);
+  }
+  gs.sync();
   return total;
+}
+
+// Same contract; kept under this name for the selection code that does not need the order.
+template <int NT, class KeyAt, class Out>
+__device__ __forceinline__ uint32_t group_compact_ge_unordered(KeyAt key_at, uint32_t n, uint64_t T,
+                                                               Out out, uint32_t rank,
+                                                               GroupScratch<NT>& sc,
+                                                               const GroupSync<NT>& gs) {
+  return group_compact_ge<NT>(key_at, n, T, out, rank, sc, gs);
+}
+
+// Descending compare-exchange of a 64-bit pair held by one thread.
+__device__ __forceinline__ void cx_desc(uint64_t& a, uint64_t& b, bool desc) {
+  const uint64_t hi = a > b ? a : b, lo = a > b ? b : a;
+  a = desc ? hi : lo;
+  b = desc ? lo : hi;
+}
+
+// One bitonic stage (size, stride known at compile time) over 16 * NT keys held 16 per thread:
+// element i = rank * 16 + r lives in v[r]. Strides below 16 stay in registers, strides up to
+// 256 exchange with warp shuffles, larger strides through xbuf (16 * NT keys).
+template <int NT, int SIZE, int STRIDE>
+__device__ __forceinline__ void bitonic_stage(uint64_t (&v)[16], uint32_t rank, uint64_t* xbuf,
+                                              const GroupSync<NT>& gs) {
+  if constexpr (STRIDE < 16) {
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      if ((r & STRIDE) == 0) {
+        const bool desc = (SIZE < 16) ? ((r & SIZE) == 0) : ((rank & (SIZE >> 4)) == 0);
+        cx_desc(v[r], v[r | STRIDE], desc);
+      }
+    }
+  } else {
+    const bool desc = ((rank & (SIZE >> 4)) == 0);
+    const bool lower = ((rank & (STRIDE >> 4)) == 0);
+    const bool keep_max = (lower == desc);
+    if constexpr (STRIDE <= 256) {
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        const uint64_t o = __shfl_xor_sync(0xFFFFFFFFu, v[r], STRIDE >> 4);
+        v[r] = keep_max ? (v[r] > o ? v[r] : o) : (v[r] > o ? o : v[r]);
+      }
+    } else {
+#pragma unroll
+      for (int r = 0; r < 16; ++r) xbuf[r * NT + rank] = v[r];
+      gs.sync();
+      const uint32_t partner = rank ^ (STRIDE >> 4);
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        const uint64_t o = xbuf[r * NT + partner];
+        v[r] = keep_max ? (v[r] > o ? v[r] : o) : (v[r] > o ? o : v[r]);
+      }
+      gs.sync();
+    }
+  }
+}
+
+template <int NT, int SIZE, int STRIDE>
+__device__ __forceinline__ void bitonic_merge_stages(uint64_t (&v)[16], uint32_t rank, uint64_t* xbuf,
+                                                     const GroupSync<NT>& gs) {
+  bitonic_stage<NT, SIZE, STRIDE>(v, rank, xbuf, gs);
+  if constexpr (STRIDE > 1) bitonic_merge_stages<NT, SIZE, STRIDE / 2>(v, rank, xbuf, gs);
+}
+
+template <int NT, int SIZE>
+__device__ __forceinline__ void bitonic_sizes(uint64_t (&v)[16], uint32_t rank, uint64_t* xbuf,
+                                              const GroupSync<NT>& gs) {
+  bitonic_merge_stages<NT, SIZE, SIZE / 2>(v, rank, xbuf, gs);
+  if constexpr (SIZE < 16 * NT) bitonic_sizes<NT, SIZE * 2>(v, rank, xbuf, gs);
+}
+
+// Sorts the 16 * NT keys held 16 per thread into descending order: afterwards thread `rank`
+// holds elements rank * 16 .. rank * 16 + 15 of the sorted sequence in v[0..15].
+template <int NT>
+__device__ void group_bitonic_sort_regs(uint64_t (&v)[16], uint32_t rank, uint64_t* xbuf,
+                                        const GroupSync<NT>& gs) {
+  static_assert(NT <= 512, "exchange strides");
+  bitonic_sizes<NT, 2>(v, rank, xbuf, gs);
 }
 
 // Sorts the 16 keys of one thread in descending order (bitonic network, fully unrolled).
@@ -210,10 +329,17 @@ __device__ __forceinline__ void sort16_desc(uint64_t (&v)[16]) {
   }
 }
 
+// Smallest power of two >= max(k, 16): the size the merge sort works on.
+__device__ __forceinline__ uint32_t sort_size(uint32_t k) {
+  uint32_t p = 16;
+  while (p < k) p <<= 1;
+  return p;
+}
+
 // Shared-memory index of element x of a sort buffer: one padding slot after every 16 keys,
 // so that the 16-key runs of consecutive threads fall into different banks.
 __device__ __forceinline__ uint32_t spad(uint32_t x) { return x + (x >> 4); }
-constexpr int sort_buffer_len(int P) { return P + P / 16; }
+__host__ __device__ constexpr int sort_buffer_len(int P) { return P + P / 16; }
 
 // Sorts P keys (P a power of two, 16 <= P <= 16 * NT) in descending order. load(e) supplies
 // key e (e < P). Each of the first P/16 threads loads 16 keys with a coalesced stride, sorts

@@ -1,50 +1,97 @@
 // Top-k finishing kernels.
-//   sort_rows_kernel   : orders each row's exact top-k keys (prefill winners) by key
-//                        descending = (score descending, index ascending) and writes
-//                        out_idx / out_score with -1 / -inf padding.
-//   decode_topk_kernel : per request, exact top-k of its n_b stored scores. The scoring kernel
-//                        has already counted the request's scores in 2048 bins of their
-//                        order-preserving top 11 bits; the bin holding the k-th score bounds
-//                        the candidates, which one pass over the scores collects into shared
-//                        memory. An exact radix select there and a merge sort finish the row.
+//   prefill_finish_kernel : per prefill query, the exact top-k of the candidate buffer the
+//                           fused scoring kernel left (four warp segments), ordered by
+//                           (score descending, index ascending) and padded with -1 / -inf.
+//   decode_topk_kernel    : per request, exact top-k of its n_b stored scores. The scoring
+//                           kernel has already counted the request's scores in 2048 bins of
+//                           their order-preserving top 11 bits; the bin holding the k-th score
+//                           bounds the candidates, which one pass over the scores collects into
+//                           shared memory. An exact radix select there and a merge sort finish
+//                           the row, in the same order and padding.
 #include "common.cuh"
 #include "internal.h"
 #include "select.cuh"
 
 namespace dsa {
 
-__device__ __forceinline__ uint32_t sort_size(uint32_t k) {
-  uint32_t p = 16;
-  while (p < k) p <<= 1;
-  return p;
-}
-
-constexpr int kSortThreads = 128;
 constexpr int kSortBuf = sort_buffer_len(DSA_MAX_TOPK);
 
-__global__ void __launch_bounds__(kSortThreads)
-    sort_rows_kernel(const uint64_t* __restrict__ win, int topk, int32_t* __restrict__ out_idx,
-                     float* __restrict__ out_score) {
-  __shared__ uint64_t a[kSortBuf];
-  __shared__ uint64_t b[kSortBuf];
-  const GroupSync<kSortThreads> gs{0};
+constexpr int kFinishThreads = 256;
+
+struct FinishSmem {
+  uint64_t stage[kPrefillCapMax];   // the row's candidates; later the two sort buffers
+  uint64_t win[DSA_MAX_TOPK];       // the k winners, contiguous
+  uint32_t hist[kHistBins];
+  GroupScratch<kFinishThreads> sc;
+};
+static_assert(kPrefillCapMax >= 2u * static_cast<uint32_t>(kSortBuf), "sort buffers in the stage");
+
+__global__ void __launch_bounds__(kFinishThreads)
+    prefill_finish_kernel(const uint64_t* __restrict__ cand, const uint32_t* __restrict__ counts,
+                          uint32_t cap, int topk, int32_t* __restrict__ out_idx,
+                          float* __restrict__ out_score) {
+  extern __shared__ uint8_t smem_raw[];
+  FinishSmem& sm = *reinterpret_cast<FinishSmem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 15) & ~static_cast<uintptr_t>(15));
+  const GroupSync<kFinishThreads> gs{0};
   const uint32_t rank = threadIdx.x;
   const size_t row = blockIdx.x;
   const uint32_t k = static_cast<uint32_t>(topk);
-  const uint32_t P = sort_size(k);
-  const uint64_t* src = win + row * k;
-  const uint64_t* s = group_merge_sort_desc<kSortThreads>(
-      [&](uint32_t e) { return e < k ? __ldcs(src + e) : 0ull; }, a, b, P, rank, gs);
-  for (uint32_t e = rank; e < k; e += kSortThreads) {
-    const uint64_t key = s[spad(e)];
-    out_idx[row * k + e] = key_index(key);
-    if (out_score) out_score[row * k + e] = key_score(key);
+  const uint32_t segcap = cap / 4u;
+  const uint64_t* buf = cand + row * cap;
+  uint32_t c[4], n = 0;
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    const uint32_t v = __ldcg(counts + row * 4 + w);
+    c[w] = v < segcap ? v : segcap;
+    n += c[w];
+  }
+  // Stage the four segments contiguously, four independent loads in flight per thread.
+  const uint32_t o1 = c[0], o2 = o1 + c[1], o3 = o2 + c[2];
+  auto src_of = [&](uint32_t e) -> const uint64_t* {
+    const uint32_t w = (e >= o1 ? 1u : 0u) + (e >= o2 ? 1u : 0u) + (e >= o3 ? 1u : 0u);
+    const uint32_t start = e >= o3 ? o3 : (e >= o2 ? o2 : (e >= o1 ? o1 : 0u));
+    return buf + w * segcap + (e - start);
+  };
+  uint32_t e = rank;
+  for (; e + 3 * kFinishThreads < n; e += 4 * kFinishThreads) {
+    const uint64_t a0 = __ldcg(src_of(e)), a1 = __ldcg(src_of(e + kFinishThreads)),
+                   a2 = __ldcg(src_of(e + 2 * kFinishThreads)), a3 = __ldcg(src_of(e + 3 * kFinishThreads));
+    sm.stage[e] = a0;
+    sm.stage[e + kFinishThreads] = a1;
+    sm.stage[e + 2 * kFinishThreads] = a2;
+    sm.stage[e + 3 * kFinishThreads] = a3;
+  }
+  for (; e < n; e += kFinishThreads) sm.stage[e] = __ldcg(src_of(e));
+  for (uint32_t b = rank; b < kHistBins; b += kFinishThreads) sm.hist[b] = 0u;
+  gs.sync();
+  auto key_at = [&](uint32_t i) { return sm.stage[i]; };
+  const uint64_t T = n > k ? group_kth_threshold<kFinishThreads>(key_at, n, k, rank, sm.hist, sm.sc, gs)
+                           : 0ull;
+  uint32_t n_win = group_compact_ge<kFinishThreads>(
+      key_at, n, T, [&](uint32_t pos, uint64_t key) { if (pos < k) sm.win[pos] = key; }, rank, sm.sc, gs);
+  n_win = n_win < k ? n_win : k;
+  const uint64_t* s = group_merge_sort_desc<kFinishThreads>(
+      [&](uint32_t i) { return i < n_win ? sm.win[i] : 0ull; }, sm.stage, sm.stage + kSortBuf,
+      sort_size(k), rank, gs);
+  int32_t* oi = out_idx + row * k;
+  float* os = out_score ? out_score + row * k : nullptr;
+  for (uint32_t i = rank; i < k; i += kFinishThreads) {
+    const uint64_t key = s[spad(i)];
+    oi[i] = key_index(key);
+    if (os) os[i] = key_score(key);
   }
 }
 
-dsa_status launch_sort_rows(const uint64_t* win, int rows, int topk, int32_t* out_idx,
-                            float* out_score, cudaStream_t stream) {
-  sort_rows_kernel<<<rows, kSortThreads, 0, stream>>>(win, topk, out_idx, out_score);
+dsa_status launch_prefill_finish(const uint64_t* cand, const uint32_t* counts, uint32_t cap,
+                                 int rows, int topk, int32_t* out_idx, float* out_score,
+                                 cudaStream_t stream) {
+  const size_t smem = sizeof(FinishSmem) + 16;
+  if (cudaFuncSetAttribute(prefill_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  prefill_finish_kernel<<<rows, kFinishThreads, smem, stream>>>(cand, counts, cap, topk, out_idx,
+                                                                out_score);
   return cuda_status(cudaGetLastError());
 }
 
@@ -106,6 +153,8 @@ __global__ void __launch_bounds__(kDecodeTopkThreads)
     gs.sync();
     const uint32_t bstar = sm.sc.w[kDecodeTopkThreads / 32];
     const uint32_t n_cand = sm.sc.w[kDecodeTopkThreads / 32 + 1];
+    gs.sync();
+    for (uint32_t b = rank; b < kHistBins; b += kDecodeTopkThreads) sm.hist[b] = 0u;  // selects below need it zero
     gs.sync();
     uint64_t T;
     if (n_cand <= kDecodeCandCap) {
