@@ -61,7 +61,7 @@ dsa_status check_decode(const uint8_t* q, const float* q_scale, const float* w,
 }  // namespace
 
 bool encode_tmap_2d_u8(CUtensorMap* map, const void* base, uint64_t row_bytes, uint64_t rows,
-                       uint32_t box_rows) {
+                       uint32_t box_rows, uint64_t row_stride) {
   static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   if (!encode) {
     void* fn = nullptr;
@@ -72,7 +72,7 @@ bool encode_tmap_2d_u8(CUtensorMap* map, const void* base, uint64_t row_bytes, u
     encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
   }
   const cuuint64_t dims[2] = {row_bytes, rows};
-  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint64_t strides[1] = {row_stride ? row_stride : row_bytes};
   const cuuint32_t box[2] = {static_cast<cuuint32_t>(row_bytes), box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUtensorMapSwizzle swz =

@@ -46,13 +46,44 @@ struct DecodeLaunch {
   int num_sms;
 };
 
-// Candidate-buffer capacity (entries) per query of the streaming prefill top-k: four warp
-// segments of cap/4 entries. A segment is cut back as soon as it holds more than cap/4 - 32
-// keys (a tile adds at most 32), and a cut-back leaves at most (k + 131) / 4 keys in it.
-__host__ __device__ constexpr uint32_t prefill_cand_cap(int topk) {
+// Prefill workspace layout. Every query row owns 4 * seg_stride candidate entries: four warp
+// segments, seg_stride entries apart. The lean pass may fill a segment up to lean_segcap
+// (about 3k/4 + 128: it expects k + 6.5 sqrt(k S) keys per row), the exact pass up to
+// exact_segcap (k/2 + 128: its cut-backs leave at most (k + 131) / 4 per segment), and the
+// sample pass up to seg_stride.
+struct PrefillLayout {
+  uint32_t seg_stride, lean_segcap, exact_segcap;
+  size_t cand_off, thr_off, counts_off, flags_off, list_off, count_off, total;
+};
+__host__ __device__ constexpr uint32_t prefill_exact_cap(int topk) {
   return (2u * static_cast<uint32_t>(topk) + 512u + 127u) & ~127u;
 }
-constexpr uint32_t kPrefillCapMax = prefill_cand_cap(DSA_MAX_TOPK);
+constexpr uint32_t kPrefillExactCapMax = prefill_exact_cap(DSA_MAX_TOPK);
+inline PrefillLayout prefill_layout(int Lq, int topk) {
+  PrefillLayout L{};
+  const uint32_t lean_cap = (3u * static_cast<uint32_t>(topk) + 512u + 127u) & ~127u;
+  const uint32_t pitch = lean_cap > prefill_exact_cap(topk) ? lean_cap : prefill_exact_cap(topk);
+  L.seg_stride = pitch / 4u;
+  L.lean_segcap = lean_cap / 4u;
+  L.exact_segcap = prefill_exact_cap(topk) / 4u;
+  const size_t rows = static_cast<size_t>(Lq);
+  const size_t nqb = rows;  // at least one flag / list slot per row covers every block size
+  size_t off = DSA_WS_HEADER_BYTES;
+  L.cand_off = off;
+  off += rows * pitch * sizeof(uint64_t);
+  L.thr_off = off;
+  off += rows * sizeof(uint64_t);
+  L.counts_off = off;
+  off += rows * 4 * sizeof(uint32_t);
+  L.flags_off = off;
+  off += nqb * sizeof(uint32_t);
+  L.list_off = off;
+  off += nqb * sizeof(int32_t);
+  L.count_off = off;
+  off += 16;
+  L.total = off;
+  return L;
+}
 inline int prefill_queries_per_block(int H) { return 2 * (256 / H); }
 
 size_t prefill_workspace_bytes(int Lq, int H, int d, int topk, int num_sms);
@@ -60,9 +91,13 @@ size_t decode_workspace_bytes(int B, int max_len, int H, int d, int topk);
 
 dsa_status launch_prefill(const PrefillLaunch& a);
 // Exact top-k of every row's candidate buffer, ordered and written to out_idx / out_score.
-dsa_status launch_prefill_finish(const uint64_t* cand, const uint32_t* counts, uint32_t cap,
-                                 int rows, int topk, int32_t* out_idx, float* out_score,
-                                 cudaStream_t stream);
+dsa_status launch_prefill_finish(const uint64_t* cand, const uint32_t* counts,
+                                 const uint64_t* thr, uint32_t pitch, int rows, int topk,
+                                 int32_t* out_idx, float* out_score, cudaStream_t stream);
+// Per prefill row, the threshold of the lean pass from the row's sampled keys.
+dsa_status launch_prefill_sample_threshold(const uint64_t* cand, const uint32_t* counts,
+                                           uint64_t* thr, uint32_t seg_stride, int rows,
+                                           int q_pos0, int Lk, int topk, cudaStream_t stream);
 dsa_status launch_decode(const DecodeLaunch& a);
 dsa_status launch_decode_topk(const float* scores, int max_len, const int32_t* seq_lens,
                               const uint32_t* bins, int B, int topk, int32_t* out_idx,
@@ -73,8 +108,9 @@ dsa_status launch_overlap(const int32_t* const* layer_idx, int32_t n_layers, int
 dsa_status launch_selftest_wait(void* ws, uint64_t budget_ns, cudaStream_t stream);
 
 // Tensor-map encoding through the driver entry point (no link-time libcuda dependency).
+// Rows of row_bytes bytes, row_stride bytes apart (0: packed), boxes of box_rows rows.
 bool encode_tmap_2d_u8(CUtensorMap* map, const void* base, uint64_t row_bytes, uint64_t rows,
-                       uint32_t box_rows);
+                       uint32_t box_rows, uint64_t row_stride = 0);
 
 inline dsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
 

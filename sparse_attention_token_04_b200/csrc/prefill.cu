@@ -1,7 +1,7 @@
-// Fused prefill lightning indexer for sm_100a: scores every causal (query, key) pair on the
-// tensor cores and streams, per query, the keys that can still enter its top-k into that
-// query's candidate buffer in the workspace. prefill_finish_kernel (topk.cu) then takes the
-// exact top-k of each buffer. The L x L score matrix is never stored.
+// Prefill lightning indexer for sm_100a: scores every causal (query, key) pair on the tensor
+// cores and streams, per query, the keys that can still enter its top-k into that query's
+// candidate buffer in the workspace; prefill_finish_kernel (topk.cu) then takes the exact top-k
+// of each buffer. The L x L score matrix is never stored.
 //
 // One persistent CTA per SM walks query blocks (heaviest first, snake order over CTAs). For a
 // block of QB queries it streams the causal key range in tiles of 128 keys:
@@ -12,13 +12,22 @@
 //               256-column accumulators so the epilogue of one overlaps the MMA of the other;
 //   warps 4-11  two epilogue warpgroups, one per accumulator. Thread = key (its TMEM lane):
 //               it reads the key's H head dot products of each query, applies ReLU, the head
-//               weights, then the query and key scales, masks s > t, and appends the keys at
-//               or above the query's threshold to its warp's segment of the query's buffer
-//               (no atomics: the segment's count lives in a register of the warp).
-// When a segment may overflow on the next tile, the warpgroup cuts that query's buffer back to
-// the keys at or above the histogram bin holding its k-th key (k to k + 128 keys), spread
-// evenly over the four segments, and raises the query's threshold to that bin's lower edge.
-// A key below the threshold has k buffered keys above it, so dropping it is exact.
+//               weights, then the query and key scales, masks s > t, and appends the keys it
+//               keeps to its warp's segment of the query's buffer (no atomics: the segment's
+//               count lives in a register of the warp).
+//
+// The same kernel runs in three modes:
+//   sample  every S-th key only (a strided tensor map), every valid key appended: a uniform
+//           sample of each row, from which prefill_sample_threshold_kernel picks a threshold T
+//           that at least k keys of the row exceed with overwhelming probability;
+//   lean    every key, appended iff key >= T: a compare and an append, nothing else. A query
+//           that ends with fewer than min(k, keys in its row) appended keys (T was too high)
+//           or a full segment marks its block for the exact mode;
+//   exact   no threshold to start with: a nearly full buffer is cut back, by the four warps
+//           together, to the keys at or above the bin holding its k-th key (k to k + 128 keys),
+//           which also raises the query's threshold. Any key below the threshold has k kept
+//           keys above it, so dropping it is exact. Runs on the blocks the lean mode marked,
+//           or on every block when k is too small for a useful sample.
 //
 // ReLU on the FMA pipe: D = q8.k8 with |D| <= d * 448^2 < 2^25, so
 // max(D, 0) = 2^25 * sat(D * 2^-25) exactly (power-of-two scalings, no clipping at 1), and
@@ -46,11 +55,13 @@ struct PCfg {
   static_assert(H == 8 || H == 64, "H");
 };
 
-// Selection state of one epilogue warpgroup's cut-backs.
+enum : int { kModeSample = 0, kModeLean = 1, kModeExact = 2 };
+
+// Selection state of one epilogue warpgroup's cut-backs (exact mode).
 struct __align__(16) CutState {
-  uint32_t hist[kHistBins];         // zero between cut-backs
+  uint32_t hist[kHistBins];             // zero between cut-backs
   GroupScratch<128> sc;
-  uint64_t stage[kPrefillCapMax];   // the buffer being cut, contiguous
+  uint64_t stage[kPrefillExactCapMax];  // the buffer being cut, contiguous
 };
 
 template <int H, int D>
@@ -60,9 +71,9 @@ struct PSmem {
   uint8_t k[C::STAGES][C::KTILE];
   float wq[C::QB][H];
   float sq[C::QB];
-  uint64_t thr[C::QB];
-  uint32_t wcnt[C::QB][4];  // per query: keys in each warp's segment, exchanged at cut-backs
-  uint32_t cflag[2];        // per warpgroup: queries whose buffer needs a cut-back
+  uint64_t thr[C::QB];      // per query: lean T; exact running threshold
+  uint32_t wcnt[C::QB][4];  // per query: keys in each warp's segment (block end, cut-backs)
+  uint32_t cflag[2];        // per warpgroup: queries whose buffer needs a cut-back (exact)
   CutState cut[2];
   uint64_t kfull[C::STAGES];
   uint64_t kempty[C::STAGES];
@@ -84,20 +95,28 @@ struct PrefillParams {
   const float* k_scale;
   int32_t Lk, q_pos0, Lq, topk;
   int32_t nqb;
-  uint32_t cap;        // candidate entries per row: four segments of cap / 4
-  uint64_t* cand;      // [Lq][cap]
-  uint32_t* counts;    // [Lq][4] keys in each segment after the scan
+  int32_t stride;          // key stride S (sample mode: map row v is key S * v), else 1
+  int32_t nkeys;           // rows of the key tensor map (sample mode: ceil(Lk / S))
+  uint32_t seg_stride;     // entries between a row's segments (row pitch / 4)
+  uint32_t segcap;         // entries a segment may hold in this mode
+  uint64_t* cand;          // [Lq][4 * seg_stride]
+  uint32_t* counts;        // [Lq][4] keys in each segment after the scan
+  uint64_t* thr;           // [Lq] lean: input T; exact: output threshold
+  uint32_t* fail_flag;     // [nqb] lean: block needs the exact mode
+  int32_t* fail_list;      // [nqb] lean: output list; exact: input list (nullptr: every block)
+  uint32_t* fail_count;
   WsHeader* hdr;
   uint64_t budget_ns;
 };
 
 // Cut-back of one query's candidate buffer by its warpgroup (128 threads on named barrier
-// bar_id). The four segment counts are in wcnt[0..3]. Stages the segments contiguously in
-// shared memory; with more than k + 128 keys it finds the lower edge T of the histogram bin
-// holding the k-th key (k <= count(keys >= T) <= k + 128) and keeps the keys >= T, otherwise it
-// keeps every key. The kept keys are written back dealt round-robin over the four segments;
-// wcnt and (after a select) *thr are updated. One out-of-line copy serves every call site.
-__device__ __noinline__ void cut_back(uint64_t* buf, uint32_t segcap, uint32_t* wcnt,
+// bar_id). The four segment counts are in wcnt[0..3], segment w at buf + w * seg_stride.
+// Stages the segments contiguously in shared memory; with more than k + 128 keys it finds the
+// lower edge T of the histogram bin holding the k-th key (k <= count(keys >= T) <= k + 128)
+// and keeps the keys >= T, otherwise it keeps every key. The kept keys are written back dealt
+// round-robin over the four segments; wcnt and (after a select) *thr are updated. One
+// out-of-line copy serves every call site.
+__device__ __noinline__ void cut_back(uint64_t* buf, uint32_t seg_stride, uint32_t* wcnt,
                                       uint64_t* thr, CutState* cs, uint32_t k, uint32_t rank,
                                       uint32_t bar_id) {
   const GroupSync<128> gs{bar_id};
@@ -109,7 +128,7 @@ __device__ __noinline__ void cut_back(uint64_t* buf, uint32_t segcap, uint32_t* 
     n += c;
   }
   const uint32_t c = wcnt[w];
-  const uint64_t* src = buf + w * segcap;
+  const uint64_t* src = buf + w * seg_stride;
   uint64_t* st = cs->stage;
   uint32_t e = lane;
   for (; e + 96 < c; e += 128) {
@@ -130,14 +149,14 @@ __device__ __noinline__ void cut_back(uint64_t* buf, uint32_t segcap, uint32_t* 
   }
   const uint32_t kept = group_compact_ge<128>(
       key_at, n, T,
-      [buf, segcap](uint32_t pos, uint64_t key) { buf[(pos & 3u) * segcap + (pos >> 2)] = key; },
+      [buf, seg_stride](uint32_t pos, uint64_t key) { buf[(pos & 3u) * seg_stride + (pos >> 2)] = key; },
       rank, cs->sc, gs);
   if (rank < 4) wcnt[rank] = (kept + 3u - rank) >> 2;
   if (rank == 0 && T != 0) *thr = T;
   gs.sync();
 }
 
-template <int H, int D>
+template <int H, int D, int MODE>
 __global__ void __launch_bounds__(384, 1)
     prefill_indexer_kernel(const __grid_constant__ CUtensorMap tmap_q,
                            const __grid_constant__ CUtensorMap tmap_k, const PrefillParams p) {
@@ -146,6 +165,11 @@ __global__ void __launch_bounds__(384, 1)
   PSmem<H, D>& sm = *reinterpret_cast<PSmem<H, D>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31u;
+
+  // Blocks this launch processes: every block, or (exact mode after a lean pass) the listed ones.
+  const bool listed = MODE == kModeExact && p.fail_list != nullptr;
+  const int nblocks = listed ? static_cast<int>(__ldcg(p.fail_count)) : p.nqb;
+  if (nblocks <= static_cast<int>(blockIdx.x)) return;  // no block for this CTA; nothing armed yet
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -176,11 +200,13 @@ __global__ void __launch_bounds__(384, 1)
   // Heaviest query block first; snake order over CTAs balances the causal triangle.
   auto block_of = [&](int r) -> int {
     const int j = r * G + ((r & 1) ? (G - 1 - cta) : cta);
-    return j < p.nqb ? p.nqb - 1 - j : -1;
+    if (j >= nblocks) return -1;
+    return listed ? __ldcg(p.fail_list + j) : p.nqb - 1 - j;
   };
   auto ntiles_of = [&](int qb) -> int {
-    const int last_row = min(qb * C::QB + C::QB, p.Lq) - 1;
-    return (p.q_pos0 + last_row) / C::BN + 1;
+    const int last_t = p.q_pos0 + min(qb * C::QB + C::QB, p.Lq) - 1;
+    const int last_key = min(last_t / p.stride, p.nkeys - 1);
+    return last_key / C::BN + 1;
   };
 
   if (warp == 0) {
@@ -274,15 +300,16 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t wl = warp & 3u;        // TMEM lane quarter = buffer segment of this warp
     const uint32_t rank = threadIdx.x - 128u * (1u + g);
     const GroupSync<128> gs{1u + g};
-    CutState* cs = &sm.cut[g];
     const uint32_t taddr0 = tmem + g * 256 + ((wl * 32u) << 16);
     const int qbase = static_cast<int>(g) * C::QPM;
     const uint32_t k = static_cast<uint32_t>(p.topk);
-    const uint32_t segcap = p.cap / 4u;
-    const uint32_t trigger = segcap - 32u;  // above it the next tile could overflow the segment
+    const uint32_t segcap = p.segcap;
+    const size_t pitch = 4u * static_cast<size_t>(p.seg_stride);
+    const uint32_t trigger = segcap - 32u;  // exact: above it the next tile could overflow
     const uint32_t lt = (1u << lane) - 1u;
-    for (int i = rank; i < kHistBins; i += 128) cs->hist[i] = 0u;  // the selects keep it zero
-    if (rank == 0) sm.cflag[g] = 0u;
+    if constexpr (MODE == kModeExact) {
+      for (int i = rank; i < kHistBins; i += 128) sm.cut[g].hist[i] = 0u;  // the selects keep it zero
+    }
     uint32_t use = 0;
     bool ok = true;
     for (int r = 0; ok; ++r) {
@@ -297,19 +324,24 @@ __global__ void __launch_bounds__(384, 1)
       for (int qi = rank; qi < C::QPM; qi += 128) {
         const int row = row_base + qi;
         sm.sq[qbase + qi] = (row < p.Lq) ? __ldg(&p.q_scale[row]) : 0.0f;
-        sm.thr[qbase + qi] = 0;
+        sm.thr[qbase + qi] = (MODE == kModeLean && row < p.Lq) ? __ldcg(p.thr + row) : 0ull;
       }
+      if (rank == 0) sm.cflag[g] = 0u;
       gs.sync();
       uint32_t cw[C::QPM];  // keys in this warp's segment, per query (warp-uniform)
 #pragma unroll
       for (int qi = 0; qi < C::QPM; ++qi) cw[qi] = 0u;
       const int nt = ntiles_of(qb);
-      int s = static_cast<int>(wl * 32u + lane);
-      float sk_next = (s < p.Lk) ? __ldg(&p.k_scale[s]) : 0.0f;
+      int v = static_cast<int>(wl * 32u + lane);  // this thread's row of the key tensor map
+      auto scale_of = [&](int vi) {
+        return vi < p.nkeys ? __ldg(&p.k_scale[static_cast<size_t>(vi) * p.stride]) : 0.0f;
+      };
+      float sk_next = scale_of(v);
       bool good = true;
-      for (int tile = 0; tile < nt; ++tile, s += C::BN) {
+      for (int tile = 0; tile < nt; ++tile, v += C::BN) {
         const float sk = sk_next;
-        sk_next = (s + C::BN < p.Lk) ? __ldg(&p.k_scale[s + C::BN]) : 0.0f;
+        sk_next = scale_of(v + C::BN);
+        const int s = v * p.stride;  // the key's position
         const bool got = mbar_wait(&sm.accfull[g], use & 1u, ctl, DETAIL_WAIT_ACCFULL);
         good = good && got;
         __syncwarp();
@@ -376,51 +408,82 @@ __global__ void __launch_bounds__(384, 1)
         if (lane == 0) mbar_arrive(&sm.accempty[g]);
         ++use;
 
-        // Inserts into this warp's own segment: no atomics, the count lives in a register.
+        // Appends to this warp's own segment: no atomics, the count lives in a register.
         uint32_t flags = 0u;
 #pragma unroll
         for (int qi = 0; qi < C::QPM; ++qi) {
           const int row = row_base + qi;
-          const bool valid = (row < p.Lq) && (s <= p.q_pos0 + row);
+          const bool valid = (row < p.Lq) && (v < p.nkeys) && (s <= p.q_pos0 + row);
           const float score = (score_part[qi] * sm.sq[qbase + qi]) * sk;
           const uint64_t key = make_key(score, static_cast<uint32_t>(s));
-          const bool take = valid && key >= sm.thr[qbase + qi];
+          const bool take = valid && (MODE == kModeSample || key >= sm.thr[qbase + qi]);
           const uint32_t m = __ballot_sync(0xFFFFFFFFu, take);
           const uint32_t pos = cw[qi] + __popc(m & lt);
-          if (take) p.cand[static_cast<size_t>(row) * p.cap + wl * segcap + pos] = key;
+          if (take && pos < segcap) p.cand[static_cast<size_t>(row) * pitch + wl * p.seg_stride + pos] = key;
           cw[qi] += __popc(m);
-          flags |= (cw[qi] > trigger) ? (1u << qi) : 0u;
+          if constexpr (MODE == kModeExact) flags |= (cw[qi] > trigger) ? (1u << qi) : 0u;
         }
-        // One decision for the whole warpgroup: the barrier ORs the warps' requests, and the
-        // flag word written before it is visible to every warp after it.
-        if (flags && lane == 0) atomicOr(&sm.cflag[g], flags);
-        if (named_bar_or(1u + g, 128, flags != 0u)) {
-          const uint32_t mask = *reinterpret_cast<volatile uint32_t*>(&sm.cflag[g]);
-          if (lane == 0) {
+        if constexpr (MODE == kModeExact) {
+          // Cut-backs: one decision for the whole warpgroup. The barrier ORs the warps'
+          // requests, and the flag word written before it is visible to every warp after it.
+          if (flags && lane == 0) atomicOr(&sm.cflag[g], flags);
+          if (named_bar_or(1u + g, 128, flags != 0u)) {
+            const uint32_t mask = *reinterpret_cast<volatile uint32_t*>(&sm.cflag[g]);
+            if (lane == 0) {
 #pragma unroll
-            for (int qi = 0; qi < C::QPM; ++qi) sm.wcnt[qbase + qi][wl] = cw[qi];
-          }
-          gs.sync();
-          if (rank == 0) sm.cflag[g] = 0u;
+              for (int qi = 0; qi < C::QPM; ++qi) sm.wcnt[qbase + qi][wl] = cw[qi];
+            }
+            gs.sync();
+            if (rank == 0) sm.cflag[g] = 0u;
 #pragma unroll 1
-          for (int qi = 0; qi < C::QPM; ++qi) {
-            if ((mask >> qi) & 1u)
-              cut_back(p.cand + static_cast<size_t>(row_base + qi) * p.cap, segcap,
-                       sm.wcnt[qbase + qi], &sm.thr[qbase + qi], cs, k, rank, 1u + g);
-          }
+            for (int qi = 0; qi < C::QPM; ++qi) {
+              if ((mask >> qi) & 1u)
+                cut_back(p.cand + static_cast<size_t>(row_base + qi) * pitch, p.seg_stride,
+                         sm.wcnt[qbase + qi], &sm.thr[qbase + qi], &sm.cut[g], k, rank, 1u + g);
+            }
 #pragma unroll
-          for (int qi = 0; qi < C::QPM; ++qi) cw[qi] = sm.wcnt[qbase + qi][wl];
+            for (int qi = 0; qi < C::QPM; ++qi) cw[qi] = sm.wcnt[qbase + qi][wl];
+          }
         }
       }
       ok = named_bar_and(1u + g, 128, ok && good);
       if (!ok) break;
-      // The segment counts of every query of this warpgroup, for the finishing kernel.
+      // Segment counts (and thresholds) of every query of this warpgroup.
       if (lane == 0) {
 #pragma unroll
         for (int qi = 0; qi < C::QPM; ++qi) {
           const int row = row_base + qi;
           if (row < p.Lq) p.counts[static_cast<size_t>(row) * 4 + wl] = cw[qi];
+          sm.wcnt[qbase + qi][wl] = cw[qi];
         }
+      }
+      if constexpr (MODE == kModeExact) {
+        for (int qi = rank; qi < C::QPM; qi += 128) {
+          const int row = row_base + qi;
+          if (row < p.Lq) p.thr[row] = sm.thr[qbase + qi];
+        }
+      }
+      if constexpr (MODE == kModeLean) {
+        // A query whose buffer lacks some of its top-k (fewer than min(k, keys in its row)
+        // appended), or whose segment overflowed, sends its block to the exact mode.
+        gs.sync();
+        bool bad = false;
+        for (int qi = rank; qi < C::QPM; qi += 128) {
+          const int row = row_base + qi;
+          if (row >= p.Lq) continue;
+          uint32_t total = 0;
+          bool full = false;
+          for (int w = 0; w < 4; ++w) {
+            const uint32_t c = sm.wcnt[qbase + qi][w];
+            total += c;
+            full = full || c > segcap;
+          }
+          const uint32_t keys = static_cast<uint32_t>(min(p.q_pos0 + row + 1, p.Lk));
+          bad = bad || full || total < min(k, keys);
+        }
+        if (bad && atomicCAS(p.fail_flag + qb, 0u, 1u) == 0u)
+          p.fail_list[atomicAdd(p.fail_count, 1u)] = qb;
+        gs.sync();  // wcnt is rewritten for the next block
       }
     }
   }
@@ -431,25 +494,41 @@ __global__ void __launch_bounds__(384, 1)
   }
 }
 
-template <int H, int D>
-static dsa_status launch_prefill_t(const PrefillLaunch& a) {
+// Key stride S of the sample pass for top-k over rows of up to Lk keys: about k / S >= 128
+// sampled keys lie above a row's k-th largest key, and a row's sample (ceil(Lk / S) keys)
+// fits its buffer. 1 means no sample pass: every block runs in the exact mode.
+static int sample_stride(int topk, int Lk, uint32_t seg_stride) {
+  const int S = topk / 128;
+  if (S < 2) return 1;
+  const int64_t room = 4 * static_cast<int64_t>(seg_stride) - 4 * 32;  // tiles end on 32-key boundaries
+  const int min_s = static_cast<int>((static_cast<int64_t>(Lk) + room - 1) / room);
+  return S > min_s ? S : min_s;
+}
+
+template <int H, int D, int MODE>
+static dsa_status launch_mode(const CUtensorMap& tq, const CUtensorMap& tk, const PrefillParams& p,
+                              int grid, cudaStream_t stream) {
   using C = PCfg<H, D>;
   // At least half of the SM's shared memory, so that one CTA (and its 512 TMEM columns)
   // owns each SM.
   size_t smem = sizeof(PSmem<H, D>) + 1024;
   if (smem < 120 * 1024) smem = 120 * 1024;
-  auto kern = prefill_indexer_kernel<H, D>;
+  auto kern = prefill_indexer_kernel<H, D, MODE>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return DSA_ERR_CUDA;
-  CUtensorMap tq, tk;
-  if (!encode_tmap_2d_u8(&tq, a.q, D, static_cast<uint64_t>(a.Lq) * H, 256)) return DSA_ERR_CUDA;
-  if (!encode_tmap_2d_u8(&tk, a.k, D, static_cast<uint64_t>(a.Lk), 128)) return DSA_ERR_CUDA;
+  kern<<<grid, C::THREADS, smem, stream>>>(tq, tk, p);
+  return cuda_status(cudaGetLastError());
+}
 
+template <int H, int D>
+static dsa_status launch_prefill_t(const PrefillLaunch& a) {
+  using C = PCfg<H, D>;
+  const PrefillLayout L = prefill_layout(a.Lq, a.topk);
   const int nqb = (a.Lq + C::QB - 1) / C::QB;
   const int grid = nqb < a.num_sms ? nqb : a.num_sms;
   uint8_t* base = static_cast<uint8_t*>(a.ws);
-  PrefillParams p;
+  PrefillParams p{};
   p.q_scale = a.q_scale;
   p.w = a.w;
   p.k_scale = a.k_scale;
@@ -458,25 +537,60 @@ static dsa_status launch_prefill_t(const PrefillLaunch& a) {
   p.Lq = a.Lq;
   p.topk = a.topk;
   p.nqb = nqb;
-  p.cap = prefill_cand_cap(a.topk);
+  p.stride = 1;
+  p.nkeys = a.Lk;
+  p.seg_stride = L.seg_stride;
+  p.segcap = L.exact_segcap;
   p.hdr = reinterpret_cast<WsHeader*>(base);
-  p.cand = reinterpret_cast<uint64_t*>(base + DSA_WS_HEADER_BYTES);
-  p.counts = reinterpret_cast<uint32_t*>(base + DSA_WS_HEADER_BYTES +
-                                         static_cast<size_t>(a.Lq) * p.cap * sizeof(uint64_t));
+  p.cand = reinterpret_cast<uint64_t*>(base + L.cand_off);
+  p.thr = reinterpret_cast<uint64_t*>(base + L.thr_off);
+  p.counts = reinterpret_cast<uint32_t*>(base + L.counts_off);
+  p.fail_flag = reinterpret_cast<uint32_t*>(base + L.flags_off);
+  p.fail_list = reinterpret_cast<int32_t*>(base + L.list_off);
+  p.fail_count = reinterpret_cast<uint32_t*>(base + L.count_off);
   p.budget_ns = a.budget_ns;
-  kern<<<grid, C::THREADS, smem, a.stream>>>(tq, tk, p);
-  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
-  return launch_prefill_finish(p.cand, p.counts, p.cap, a.Lq, a.topk, a.out_idx, a.out_score,
-                               a.stream);
+
+  CUtensorMap tq, tk;
+  if (!encode_tmap_2d_u8(&tq, a.q, D, static_cast<uint64_t>(a.Lq) * H, 256)) return DSA_ERR_CUDA;
+  if (!encode_tmap_2d_u8(&tk, a.k, D, static_cast<uint64_t>(a.Lk), 128)) return DSA_ERR_CUDA;
+
+  const int S = sample_stride(a.topk, a.Lk, L.seg_stride);
+  dsa_status st;
+  if (S > 1) {
+    // Sample pass over keys 0, S, 2S, ...: every valid sampled key appended.
+    CUtensorMap ts;
+    const int nks = (a.Lk + S - 1) / S;
+    if (!encode_tmap_2d_u8(&ts, a.k, D, static_cast<uint64_t>(nks), 128, static_cast<uint64_t>(S) * D))
+      return DSA_ERR_CUDA;
+    PrefillParams ps = p;
+    ps.stride = S;
+    ps.nkeys = nks;
+    ps.segcap = L.seg_stride;
+    if ((st = launch_mode<H, D, kModeSample>(tq, ts, ps, grid, a.stream)) != DSA_OK) return st;
+    if ((st = launch_prefill_sample_threshold(p.cand, p.counts, p.thr, L.seg_stride, a.Lq, a.q_pos0,
+                                              a.Lk, a.topk, a.stream)) != DSA_OK)
+      return st;
+    // Lean pass with those thresholds; blocks it cannot finish are listed for the exact mode.
+    if (cudaMemsetAsync(base + L.flags_off, 0, L.total - L.flags_off, a.stream) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    PrefillParams pl = p;
+    pl.segcap = L.lean_segcap;
+    if ((st = launch_mode<H, D, kModeLean>(tq, tk, pl, grid, a.stream)) != DSA_OK) return st;
+    if ((st = launch_mode<H, D, kModeExact>(tq, tk, p, grid, a.stream)) != DSA_OK) return st;
+  } else {
+    PrefillParams pe = p;
+    pe.fail_list = nullptr;
+    if ((st = launch_mode<H, D, kModeExact>(tq, tk, pe, grid, a.stream)) != DSA_OK) return st;
+  }
+  return launch_prefill_finish(p.cand, p.counts, p.thr, 4u * L.seg_stride, a.Lq, a.topk,
+                               a.out_idx, a.out_score, a.stream);
 }
 
 size_t prefill_workspace_bytes(int Lq, int H, int d, int topk, int num_sms) {
   (void)H;
   (void)d;
   (void)num_sms;
-  const size_t cand = static_cast<size_t>(Lq) * prefill_cand_cap(topk) * sizeof(uint64_t);
-  const size_t counts = static_cast<size_t>(Lq) * 4 * sizeof(uint32_t);
-  return DSA_WS_HEADER_BYTES + cand + counts;
+  return prefill_layout(Lq, topk).total;
 }
 
 dsa_status launch_prefill(const PrefillLaunch& a) {

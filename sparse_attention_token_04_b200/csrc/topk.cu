@@ -1,7 +1,10 @@
-// Top-k finishing kernels.
+// Top-k kernels.
+//   prefill_sample_threshold_kernel : per prefill query, the lean pass's threshold from the
+//                           query's sampled keys.
 //   prefill_finish_kernel : per prefill query, the exact top-k of the candidate buffer the
-//                           fused scoring kernel left (four warp segments), ordered by
-//                           (score descending, index ascending) and padded with -1 / -inf.
+//                           fused scoring kernel left (four warp segments and a threshold),
+//                           ordered by (score descending, index ascending) and padded with
+//                           -1 / -inf.
 //   decode_topk_kernel    : per request, exact top-k of its n_b stored scores. The scoring
 //                           kernel has already counted the request's scores in 2048 bins of
 //                           their order-preserving top 11 bits; the bin holding the k-th score
@@ -16,82 +19,276 @@ namespace dsa {
 
 constexpr int kSortBuf = sort_buffer_len(DSA_MAX_TOPK);
 
-constexpr int kFinishThreads = 256;
+// Prefill finish. The keys at or above the row's threshold (normally k plus a few hundred) are
+// collected in shared memory and ranked by a bucket sort: 4096 buckets of equal width in score
+// value between the smallest and largest collected score (the rounded fp32 map is monotone, so
+// a larger key never lands in a lower bucket), a suffix scan for each bucket's first rank, and
+// inside a bucket a key's rank is found by comparing it with the bucket's other keys. Keys with rank
+// below k are the top-k in order. When a bucket holds more than kBucketMax keys (heavy ties,
+// scores bunched in a sliver of their span) the row falls back to an exact radix select and a
+// merge sort.
+constexpr int kFinishThreads = 512;
+constexpr uint32_t kFinishTmp = 4608;
+constexpr int kFinishKPT = kFinishTmp / kFinishThreads;  // keys ranked per thread
+constexpr int kFinishBuckets = 4096;
+constexpr uint32_t kBucketMax = 256;
 
 struct FinishSmem {
-  uint64_t stage[kPrefillCapMax];   // the row's candidates; later the two sort buffers
-  uint64_t win[DSA_MAX_TOPK];       // the k winners, contiguous
-  uint32_t hist[kHistBins];
+  uint64_t tmp[kFinishTmp];      // collected keys, then ranked keys; merge-sort buffers
+  uint32_t bk[kFinishBuckets];   // bucket counts, then first ranks; radix histogram, then winners
   GroupScratch<kFinishThreads> sc;
+  uint32_t n_tmp;
+  uint32_t big;
+  uint32_t omin, omax;           // order-preserving score bits of the smallest / largest key
 };
-static_assert(kPrefillCapMax >= 2u * static_cast<uint32_t>(kSortBuf), "sort buffers in the stage");
+static_assert(kFinishTmp % kFinishThreads == 0, "keys per thread");
+static_assert(kFinishTmp >= 2u * static_cast<uint32_t>(kSortBuf), "merge-sort buffers in tmp");
+static_assert(kFinishBuckets * sizeof(uint32_t) >= DSA_MAX_TOPK * sizeof(uint64_t), "winners in bk");
+static_assert(kFinishBuckets >= kHistBins, "radix histogram in bk");
 
 __global__ void __launch_bounds__(kFinishThreads)
     prefill_finish_kernel(const uint64_t* __restrict__ cand, const uint32_t* __restrict__ counts,
-                          uint32_t cap, int topk, int32_t* __restrict__ out_idx,
-                          float* __restrict__ out_score) {
+                          const uint64_t* __restrict__ thr_in, uint32_t pitch, int topk,
+                          int32_t* __restrict__ out_idx, float* __restrict__ out_score) {
   extern __shared__ uint8_t smem_raw[];
   FinishSmem& sm = *reinterpret_cast<FinishSmem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 15) & ~static_cast<uintptr_t>(15));
   const GroupSync<kFinishThreads> gs{0};
-  const uint32_t rank = threadIdx.x;
+  const uint32_t rank = threadIdx.x, lane = rank & 31u, lt = (1u << lane) - 1u;
   const size_t row = blockIdx.x;
   const uint32_t k = static_cast<uint32_t>(topk);
-  const uint32_t segcap = cap / 4u;
-  const uint64_t* buf = cand + row * cap;
-  uint32_t c[4], n = 0;
+  const uint32_t segcap = pitch / 4u;
+  const uint64_t* buf = cand + row * pitch;
+  uint32_t c[4];
 #pragma unroll
   for (int w = 0; w < 4; ++w) {
     const uint32_t v = __ldcg(counts + row * 4 + w);
     c[w] = v < segcap ? v : segcap;
-    n += c[w];
   }
-  // Stage the four segments contiguously, four independent loads in flight per thread.
-  const uint32_t o1 = c[0], o2 = o1 + c[1], o3 = o2 + c[2];
+  const uint32_t o1 = c[0], o2 = o1 + c[1], o3 = o2 + c[2], n = o3 + c[3];
+  const uint64_t thr = __ldcg(thr_in + row);
   auto src_of = [&](uint32_t e) -> const uint64_t* {
     const uint32_t w = (e >= o1 ? 1u : 0u) + (e >= o2 ? 1u : 0u) + (e >= o3 ? 1u : 0u);
     const uint32_t start = e >= o3 ? o3 : (e >= o2 ? o2 : (e >= o1 ? o1 : 0u));
     return buf + w * segcap + (e - start);
   };
-  uint32_t e = rank;
-  for (; e + 3 * kFinishThreads < n; e += 4 * kFinishThreads) {
-    const uint64_t a0 = __ldcg(src_of(e)), a1 = __ldcg(src_of(e + kFinishThreads)),
-                   a2 = __ldcg(src_of(e + 2 * kFinishThreads)), a3 = __ldcg(src_of(e + 3 * kFinishThreads));
-    sm.stage[e] = a0;
-    sm.stage[e + kFinishThreads] = a1;
-    sm.stage[e + 2 * kFinishThreads] = a2;
-    sm.stage[e + 3 * kFinishThreads] = a3;
+  for (uint32_t b = rank; b < kFinishBuckets; b += kFinishThreads) sm.bk[b] = 0u;
+  if (rank == 0) {
+    sm.n_tmp = 0u;
+    sm.big = 0u;
+    sm.omin = 0xFFFFFFFFu;
+    sm.omax = 0u;
   }
-  for (; e < n; e += kFinishThreads) sm.stage[e] = __ldcg(src_of(e));
-  for (uint32_t b = rank; b < kHistBins; b += kFinishThreads) sm.hist[b] = 0u;
   gs.sync();
-  auto key_at = [&](uint32_t i) { return sm.stage[i]; };
-  const uint64_t T = n > k ? group_kth_threshold<kFinishThreads>(key_at, n, k, rank, sm.hist, sm.sc, gs)
-                           : 0ull;
-  uint32_t n_win = group_compact_ge<kFinishThreads>(
-      key_at, n, T, [&](uint32_t pos, uint64_t key) { if (pos < k) sm.win[pos] = key; }, rank, sm.sc, gs);
-  n_win = n_win < k ? n_win : k;
-  const uint64_t* s = group_merge_sort_desc<kFinishThreads>(
-      [&](uint32_t i) { return i < n_win ? sm.win[i] : 0ull; }, sm.stage, sm.stage + kSortBuf,
-      sort_size(k), rank, gs);
+  // Collect the keys at or above the threshold, sixteen independent loads in flight per thread
+  // (the whole buffer in one round for up to 8192 entries), with their score range.
+  uint32_t lmin = 0xFFFFFFFFu, lmax = 0u;
+  for (uint32_t e0 = 0; e0 < n; e0 += 16 * kFinishThreads) {
+    uint64_t v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t e = e0 + i * kFinishThreads + rank;
+      v[i] = e < n ? __ldcg(src_of(e)) : 0ull;
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const bool take = v[i] != 0ull && v[i] >= thr;
+      const uint32_t mm = __ballot_sync(0xFFFFFFFFu, take);
+      if (mm) {
+        uint32_t base = 0;
+        if (lane == 0) base = atomicAdd(&sm.n_tmp, static_cast<uint32_t>(__popc(mm)));
+        base = __shfl_sync(0xFFFFFFFFu, base, 0);
+        const uint32_t pos = base + __popc(mm & lt);
+        if (take && pos < kFinishTmp) sm.tmp[pos] = v[i];
+        if (take) {
+          const uint32_t o = static_cast<uint32_t>(v[i] >> 32);
+          lmin = o < lmin ? o : lmin;
+          lmax = o > lmax ? o : lmax;
+        }
+      }
+    }
+  }
+  lmin = __reduce_min_sync(0xFFFFFFFFu, lmin);
+  lmax = __reduce_max_sync(0xFFFFFFFFu, lmax);
+  if (lane == 0 && lmax != 0u) {
+    atomicMin(&sm.omin, lmin);
+    atomicMax(&sm.omax, lmax);
+  }
+  gs.sync();
+  const uint32_t m = sm.n_tmp;
+  const uint64_t* res = sm.tmp;
+  bool padded = false;
+  uint32_t n_res = 0;
+  bool need_select = m > kFinishTmp;
+  auto tmp_at = [&](uint32_t i) { return sm.tmp[i]; };
+  if (!need_select && m > 0) {
+    const float smin = ordered_to_float(sm.omin), smax = ordered_to_float(sm.omax);
+    const float span = smax - smin;
+    // Buckets of equal width in score; a zero (or overflowing) span puts every key in bucket 0.
+    const float scale = (span > 0.0f && span < 3.0e38f) ? (kFinishBuckets - 0.5f) / span : 0.0f;
+    uint64_t v[kFinishKPT];
+    uint32_t bs[kFinishKPT];  // bucket << 16 | slot in the bucket
+#pragma unroll
+    for (int i = 0; i < kFinishKPT; ++i) {
+      const uint32_t e = rank + i * kFinishThreads;
+      v[i] = 0ull;
+      bs[i] = 0u;
+      if (e < m) {
+        v[i] = sm.tmp[e];
+        const float f = (key_score(v[i]) - smin) * scale;
+        const uint32_t b = min(static_cast<uint32_t>(f > 0.0f ? f : 0.0f), static_cast<uint32_t>(kFinishBuckets - 1));
+        const uint32_t slot = atomicAdd(&sm.bk[b], 1u);
+        bs[i] = (b << 16) | slot;
+        if (slot >= kBucketMax) sm.big = 1u;
+      }
+    }
+    gs.sync();
+    if (sm.big) {
+      need_select = true;
+      for (uint32_t b = rank; b < kFinishBuckets; b += kFinishThreads) sm.bk[b] = 0u;
+      gs.sync();
+    } else {
+      // First rank of each bucket: keys in higher buckets (exclusive suffix sum), in place.
+      constexpr int BPT = kFinishBuckets / kFinishThreads;
+      uint32_t cnt[BPT];
+      uint32_t local = 0;
+#pragma unroll
+      for (int i = 0; i < BPT; ++i) {
+        cnt[i] = sm.bk[rank * BPT + i];
+        local += cnt[i];
+      }
+      uint32_t acc = group_suffix_exclusive<kFinishThreads>(local, rank, sm.sc.w, gs, nullptr);
+#pragma unroll
+      for (int i = BPT - 1; i >= 0; --i) {
+        sm.bk[rank * BPT + i] = acc;
+        acc += cnt[i];
+      }
+      gs.sync();
+      // Bucket members side by side (every key is in registers by now).
+#pragma unroll
+      for (int i = 0; i < kFinishKPT; ++i) {
+        const uint32_t e = rank + i * kFinishThreads;
+        if (e < m) sm.tmp[sm.bk[bs[i] >> 16] + (bs[i] & 0xFFFFu)] = v[i];
+      }
+      gs.sync();
+      // Rank = first rank of the bucket + members of the bucket that are larger.
+#pragma unroll
+      for (int i = 0; i < kFinishKPT; ++i) {
+        const uint32_t e = rank + i * kFinishThreads;
+        if (e < m) {
+          const uint32_t b = bs[i] >> 16;
+          const uint32_t s0 = sm.bk[b];
+          const uint32_t nb = (b == 0 ? m : sm.bk[b - 1]) - s0;
+          uint32_t r = s0;
+          for (uint32_t j = 0; j < nb; ++j) r += sm.tmp[s0 + j] > v[i] ? 1u : 0u;
+          bs[i] = r;
+        }
+      }
+      gs.sync();
+#pragma unroll
+      for (int i = 0; i < kFinishKPT; ++i) {
+        const uint32_t e = rank + i * kFinishThreads;
+        if (e < m && bs[i] < k) sm.tmp[bs[i]] = v[i];
+      }
+      gs.sync();
+      n_res = m < k ? m : k;
+    }
+  }
+  if (need_select) {
+    // Exact radix select of the k-th key and a merge sort of the winners. bk is zero here.
+    uint64_t* win = reinterpret_cast<uint64_t*>(sm.bk);
+    uint32_t nw;
+    if (m <= kFinishTmp) {
+      const uint64_t T = m > k ? group_kth_threshold<kFinishThreads>(tmp_at, m, k, rank, sm.bk, sm.sc, gs) : 0ull;
+      nw = group_compact_ge<kFinishThreads>(
+          tmp_at, m, T, [&](uint32_t pos, uint64_t key) { if (pos < k) win[pos] = key; }, rank, sm.sc, gs);
+    } else {
+      auto key_at = [&](uint32_t e) {
+        const uint64_t v = __ldcg(src_of(e));
+        return v >= thr ? v : 0ull;
+      };
+      const uint64_t T = group_kth_threshold<kFinishThreads>(key_at, n, k, rank, sm.bk, sm.sc, gs);
+      nw = group_compact_ge<kFinishThreads>(
+          key_at, n, T, [&](uint32_t pos, uint64_t key) { if (pos < k) win[pos] = key; }, rank, sm.sc, gs);
+    }
+    nw = nw < k ? nw : k;
+    res = group_merge_sort_desc<kFinishThreads>(
+        [&](uint32_t i) { return i < nw ? win[i] : 0ull; }, sm.tmp, sm.tmp + kSortBuf, sort_size(k),
+        rank, gs);
+    padded = true;
+    n_res = nw;
+  }
   int32_t* oi = out_idx + row * k;
   float* os = out_score ? out_score + row * k : nullptr;
   for (uint32_t i = rank; i < k; i += kFinishThreads) {
-    const uint64_t key = s[spad(i)];
+    const uint64_t key = i < n_res ? res[padded ? spad(i) : i] : 0ull;
     oi[i] = key_index(key);
     if (os) os[i] = key_score(key);
   }
 }
 
-dsa_status launch_prefill_finish(const uint64_t* cand, const uint32_t* counts, uint32_t cap,
-                                 int rows, int topk, int32_t* out_idx, float* out_score,
-                                 cudaStream_t stream) {
+dsa_status launch_prefill_finish(const uint64_t* cand, const uint32_t* counts,
+                                 const uint64_t* thr, uint32_t pitch, int rows, int topk,
+                                 int32_t* out_idx, float* out_score, cudaStream_t stream) {
   const size_t smem = sizeof(FinishSmem) + 16;
   if (cudaFuncSetAttribute(prefill_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return DSA_ERR_CUDA;
-  prefill_finish_kernel<<<rows, kFinishThreads, smem, stream>>>(cand, counts, cap, topk, out_idx,
-                                                                out_score);
+  prefill_finish_kernel<<<rows, kFinishThreads, smem, stream>>>(cand, counts, thr, pitch, topk,
+                                                                out_idx, out_score);
+  return cuda_status(cudaGetLastError());
+}
+
+// Lean-pass threshold of one prefill query from a uniform sample of its keys. The query's row
+// holds n keys, n_s of them sampled (four segments, seg_stride apart); about rho = k n_s / n
+// sampled keys lie above the row's k-th largest key, with a binomial spread of sqrt(rho). T is
+// the r-th largest sampled key for r = rho + 6.5 sqrt(rho) + 1: more than r sampled keys above
+// the k-th largest key is a 6.5-sigma event, and otherwise at least k keys of the row are >= T.
+// A row with r >= n_s (short rows, n <= k) gets T = 0: every key is kept. (The lean pass checks
+// the count it actually appended and hands the rare failure to the exact pass.)
+constexpr int kSampleThreads = 128;
+
+__global__ void __launch_bounds__(kSampleThreads)
+    prefill_sample_threshold_kernel(const uint64_t* __restrict__ cand, const uint32_t* __restrict__ counts,
+                                    uint64_t* __restrict__ thr, uint32_t seg_stride, int q_pos0, int Lk,
+                                    int topk) {
+  __shared__ uint32_t hist[kHistBins];
+  __shared__ GroupScratch<kSampleThreads> sc;
+  const GroupSync<kSampleThreads> gs{0};
+  const uint32_t rank = threadIdx.x;
+  const size_t row = blockIdx.x;
+  const uint64_t* buf = cand + row * 4u * seg_stride;
+  uint32_t c[4];
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    const uint32_t v = __ldcg(counts + row * 4 + w);
+    c[w] = v < seg_stride ? v : seg_stride;
+  }
+  const uint32_t o1 = c[0], o2 = o1 + c[1], o3 = o2 + c[2], ns = o3 + c[3];
+  const int keys = min(q_pos0 + static_cast<int>(row) + 1, Lk);
+  const double rho = static_cast<double>(topk) * ns / keys;
+  const double rr = rho + 6.5 * sqrt(rho) + 1.0;
+  if (rr >= static_cast<double>(ns)) {
+    if (rank == 0) thr[row] = 0ull;
+    return;
+  }
+  const uint32_t r = static_cast<uint32_t>(ceil(rr));
+  for (uint32_t b = rank; b < kHistBins; b += kSampleThreads) hist[b] = 0u;
+  gs.sync();
+  auto key_at = [&](uint32_t e) {
+    const uint32_t w = (e >= o1 ? 1u : 0u) + (e >= o2 ? 1u : 0u) + (e >= o3 ? 1u : 0u);
+    const uint32_t start = e >= o3 ? o3 : (e >= o2 ? o2 : (e >= o1 ? o1 : 0u));
+    return __ldcg(buf + w * seg_stride + (e - start));
+  };
+  const uint64_t T = group_kth_threshold<kSampleThreads>(key_at, ns, r, rank, hist, sc, gs);
+  if (rank == 0) thr[row] = T;
+}
+
+dsa_status launch_prefill_sample_threshold(const uint64_t* cand, const uint32_t* counts,
+                                           uint64_t* thr, uint32_t seg_stride, int rows,
+                                           int q_pos0, int Lk, int topk, cudaStream_t stream) {
+  prefill_sample_threshold_kernel<<<rows, kSampleThreads, 0, stream>>>(cand, counts, thr, seg_stride,
+                                                                       q_pos0, Lk, topk);
   return cuda_status(cudaGetLastError());
 }
 

@@ -16,6 +16,8 @@ from .inputs import (  # noqa: F401
     gmm_layer,
     correlated_layers,
     exact_layer,
+    ordered_stream_layer,
+    periodic_stream_layer,
     decode_lengths,
     paged_decode_layers,
     SEARCHED_QUARTER_PATTERN,

@@ -224,6 +224,47 @@ def exact_layer(L: int, H: int, d: int, seed: int, device="cpu") -> PrefillLayer
     return layer.to(device)
 
 
+def ordered_stream_layer(L: int, H: int, d: int, order: str, device="cpu") -> PrefillLayer:
+    """Key streams whose score order is fixed by construction (no randomness).
+
+    Every q and k code is E4M3 1.0, q scales are 1 and every head weight is 1/H, so each
+    head dot product equals d and the score of (t, s) is d * k_scale[s] * (sum of weights),
+    the same for every query. order = "increasing": k_scale[s] = 1 + s/1024 (strictly
+    increasing along s, exact in fp32), so every new key beats all earlier ones;
+    "decreasing": k_scale[s] = 1 + (L - s)/1024; "constant": all q codes are 0, so every
+    score is exactly 0 and only the index breaks ties.
+    """
+    one = _exact_codes(torch.ones(1))[0]
+    q = torch.full((L, H, d), int(one), dtype=torch.uint8)
+    if order == "constant":
+        q.zero_()
+    k = torch.full((L, d), int(one), dtype=torch.uint8)
+    s = torch.arange(L, dtype=torch.float64)
+    if order == "decreasing":
+        s = L - s
+    ks = (1.0 + s / 1024.0).to(torch.float32)
+    layer = PrefillLayer(q, torch.ones(L, dtype=torch.float32), torch.full((L, H), 1.0 / H, dtype=torch.float32),
+                         k, ks.contiguous())
+    return layer.to(device)
+
+
+def periodic_stream_layer(L: int, H: int, d: int, period: int, high_on_multiples: bool,
+                          device="cpu") -> PrefillLayer:
+    """Like ordered_stream_layer("increasing"), with every period-th key (s % period == 0) four
+    times as strong as the rest (high_on_multiples) or every other key four times as strong.
+
+    k_scale[s] = (1 + s/2^20) * (4 or 1), exact in fp32, so all scores are distinct and the
+    top-k order is fixed: the strong keys newest first, then the weak keys newest first.
+    """
+    layer = ordered_stream_layer(L, H, d, "increasing")
+    s = torch.arange(L, dtype=torch.float64)
+    on = (torch.arange(L) % period) == 0
+    strong = on if high_on_multiples else ~on
+    ks = (1.0 + s / 2.0 ** 20) * torch.where(strong, 4.0, 1.0).to(torch.float64)
+    layer = PrefillLayer(layer.q, layer.q_scale, layer.w, layer.k, ks.to(torch.float32).contiguous())
+    return layer.to(device)
+
+
 def decode_lengths(B: int, lo: int, hi: int, seed: int) -> List[int]:
     """Per-request cache lengths, uniform integers in [lo, hi]."""
     g = _generator(seed, "cpu")

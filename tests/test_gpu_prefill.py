@@ -112,3 +112,55 @@ def test_invalid_arguments_raise():
         B.dsa_indexer_prefill(layer.q, layer.q_scale, layer.w, layer.k[:32].contiguous(),
                               layer.k_scale[:32].contiguous(), 8)
     assert e.value.status == B.DSA_ERR_INVALID
+
+
+def _expected_ordered(order, L, topk):
+    rows = []
+    for t in range(L):
+        n = min(topk, t + 1)
+        if order == "increasing":
+            r = list(range(t, t - n, -1))
+        else:  # decreasing or constant: the lowest indices win
+            r = list(range(n))
+        rows.append(r + [-1] * (topk - n))
+    return np.array(rows, dtype=np.int32)
+
+
+@pytest.mark.parametrize("order", ["increasing", "constant", "decreasing"])
+@pytest.mark.parametrize("H,d,L,topk", [(64, 128, 9000, 2048), (64, 128, 3000, 7), (8, 64, 3000, 100)])
+def test_ordered_streams_closed_form(order, H, d, L, topk):
+    """Key streams with a known order: increasing scores append every key (buffer overflow and
+    compaction), constant scores tie everywhere (exact select on tied keys, tie order by index),
+    decreasing scores stop appending early. Every row is checked against its closed form."""
+    from synth import ordered_stream_layer
+
+    layer = ordered_stream_layer(L, H, d, order)
+    idx, sc = run_prefill(layer, topk)
+    assert np.array_equal(idx, _expected_ordered(order, L, topk))
+    ks = layer.k_scale.numpy().astype(np.float64)
+    valid = idx >= 0
+    want = np.where(valid, (0.0 if order == "constant" else d) * ks[np.maximum(idx, 0)], -np.inf)
+    assert np.allclose(sc[valid], want[valid], rtol=1e-6, atol=0)
+    assert np.all(np.isneginf(sc[~valid]))
+
+
+@pytest.mark.parametrize("high_on_multiples", [True, False])
+def test_periodic_streams_defeat_the_sample(high_on_multiples):
+    """Scores that follow the sampling period: when the sampled keys are the strong ones, the
+    sampled threshold keeps too few keys and those blocks are redone exactly; when they are the
+    weak ones, buffers take almost every key (overflowing segments late in the rows). Every row
+    is checked against the closed-form order."""
+    from synth import periodic_stream_layer
+
+    L, topk = 9000, 2048
+    layer = periodic_stream_layer(L, 64, 128, 16, high_on_multiples)
+    idx, sc = run_prefill(layer, topk)
+    ks = layer.k_scale.numpy().astype(np.float64)
+    for t in range(0, L, 7):
+        n = min(topk, t + 1)
+        order = np.lexsort((np.arange(t + 1), -ks[: t + 1]))[:n]
+        assert np.array_equal(idx[t, :n], order), t
+        assert np.all(idx[t, n:] == -1)
+    rows = [0, 5, 2047, 2048, 3300, 5000, 7200, L - 1]
+    for r in O.prefill_rows(layer.numpy(), topk, rows):
+        check_row(idx[r.t], sc[r.t], r, topk)
