@@ -49,13 +49,28 @@ struct PCfg {
   static constexpr int QTILE = 256 * D;     // bytes of one B operand
   static constexpr int KTILE = BN * D;      // bytes of one A operand
   static constexpr int KSTEPS = D / 32;     // K = 32 per FP8 MMA instruction
-  static constexpr int THREADS = 384;
-  static constexpr uint32_t IDESC = make_idesc_f8(128, 256);
   static_assert(D == 64 || D == 128, "d");
   static_assert(H == 8 || H == 64, "H");
 };
 
 enum : int { kModeSample = 0, kModeLean = 1, kModeExact = 2 };
+
+// Accumulators and warp roles per mode. The 512 TMEM columns hold NACC accumulators of
+// N = 512 / NACC columns ((N / H) queries x H heads); each accumulator is read by four epilogue
+// warps, one per TMEM lane quarter. The exact mode has two accumulators (N = 256) and 8
+// epilogue warps, so that its two warpgroups' cut-back state fits in shared memory; the sample
+// and lean modes have four (N = 128) and 16 epilogue warps: twice the warps to hide the
+// TMEM-load and arithmetic latency of the per-key work, and an accumulator's next MMA waits
+// only for its own four warps.
+template <int H, int MODE>
+struct PRoles {
+  static constexpr int NACC = MODE == kModeExact ? 2 : 4;
+  static constexpr int N = 512 / NACC;                    // MMA N (columns per accumulator)
+  static constexpr int EW = 4 * NACC;                     // epilogue warps
+  static constexpr int THREADS = 128 + 32 * EW;
+  static constexpr int QPW = N / H;                       // queries per accumulator and warp
+  static constexpr uint32_t IDESC = make_idesc_f8(128, N);
+};
 
 // Selection state of one epilogue warpgroup's cut-backs (exact mode).
 struct __align__(16) CutState {
@@ -73,11 +88,11 @@ struct PSmem {
   float sq[C::QB];
   uint64_t thr[C::QB];      // per query: lean T; exact running threshold
   uint32_t wcnt[C::QB][4];  // per query: keys in each warp's segment (block end, cut-backs)
-  uint32_t cflag[2];        // per warpgroup: queries whose buffer needs a cut-back (exact)
-  CutState cut[2];
+  uint32_t cflag[4];        // per query group: queries whose buffer needs a cut-back (exact)
+  CutState cut[2];          // per query group of the exact mode (two groups)
   uint64_t kfull[C::STAGES];
   uint64_t kempty[C::STAGES];
-  uint64_t qfull, qempty, accfull[2], accempty[2], drain;
+  uint64_t qfull, qempty, accfull[4], accempty[4], drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -157,7 +172,7 @@ __device__ __noinline__ void cut_back(uint64_t* buf, uint32_t seg_stride, uint32
 }
 
 template <int H, int D, int MODE>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(PRoles<H, MODE>::THREADS, 1)
     prefill_indexer_kernel(const __grid_constant__ CUtensorMap tmap_q,
                            const __grid_constant__ CUtensorMap tmap_k, const PrefillParams p) {
   using C = PCfg<H, D>;
@@ -178,7 +193,7 @@ __global__ void __launch_bounds__(384, 1)
     }
     mbar_init(&sm.qfull, 1);
     mbar_init(&sm.qempty, 1);
-    for (int g = 0; g < 2; ++g) {
+    for (int g = 0; g < PRoles<H, MODE>::NACC; ++g) {
       mbar_init(&sm.accfull[g], 1);
       mbar_init(&sm.accempty[g], 4);
     }
@@ -249,8 +264,11 @@ __global__ void __launch_bounds__(384, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      uint32_t gi = 0, it = 0, use0 = 0, use1 = 0;
-      const uint32_t qa0 = smem_u32(sm.q[0]), qa1 = smem_u32(sm.q[1]);
+      using R = PRoles<H, MODE>;
+      uint32_t gi = 0, it = 0;
+      uint32_t uses[R::NACC];
+      for (int g = 0; g < R::NACC; ++g) uses[g] = 0;
+      const uint32_t qa0 = smem_u32(sm.q[0]);  // the block's Q rows, R::N rows per accumulator
       bool ok = true;
       for (int r = 0; ok; ++r) {
         const int qb = block_of(r);
@@ -267,21 +285,20 @@ __global__ void __launch_bounds__(384, 1)
           tc_fence_after();
           const uint32_t ka = smem_u32(sm.k[st]);
 #pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            const uint32_t use = g ? use1 : use0;
-            if (!mbar_wait(&sm.accempty[g], (use & 1u) ^ 1u, ctl, DETAIL_WAIT_ACCEMPTY)) {
+          for (int g = 0; g < R::NACC; ++g) {
+            if (!mbar_wait(&sm.accempty[g], (uses[g] & 1u) ^ 1u, ctl, DETAIL_WAIT_ACCEMPTY)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint32_t qa = g ? qa1 : qa0;
+            const uint32_t qa = qa0 + g * (R::N * D);
 #pragma unroll
             for (int kk = 0; kk < C::KSTEPS; ++kk) {
-              tc_mma_f8(tmem + g * 256, make_smem_desc(ka + kk * 32, D),
-                        make_smem_desc(qa + kk * 32, D), C::IDESC, kk > 0 ? 1u : 0u);
+              tc_mma_f8(tmem + g * R::N, make_smem_desc(ka + kk * 32, D),
+                        make_smem_desc(qa + kk * 32, D), R::IDESC, kk > 0 ? 1u : 0u);
             }
             tc_commit(&sm.accfull[g]);
-            if (g) ++use1; else ++use0;
+            ++uses[g];
           }
           if (ok) tc_commit(&sm.kempty[st]);
         }
@@ -296,19 +313,22 @@ __global__ void __launch_bounds__(384, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------------ epilogue
-    const uint32_t g = (warp - 4) >> 2;   // accumulator / warpgroup
-    const uint32_t wl = warp & 3u;        // TMEM lane quarter = buffer segment of this warp
-    const uint32_t rank = threadIdx.x - 128u * (1u + g);
-    const GroupSync<128> gs{1u + g};
-    const uint32_t taddr0 = tmem + g * 256 + ((wl * 32u) << 16);
-    const int qbase = static_cast<int>(g) * C::QPM;
+    using R = PRoles<H, MODE>;
+    constexpr int QPW = R::QPW;
+    const uint32_t g = (warp - 4) >> 2;             // accumulator (and its query group)
+    const uint32_t sub = g;
+    const uint32_t wl = warp & 3u;                  // TMEM lane quarter = buffer segment
+    const uint32_t rank = wl * 32u + lane;          // rank within the group's 128 threads
+    const GroupSync<128> gs{1u + sub};
+    const uint32_t taddr0 = tmem + g * R::N + ((wl * 32u) << 16);
+    const int qbase = static_cast<int>(g) * QPW;
     const uint32_t k = static_cast<uint32_t>(p.topk);
     const uint32_t segcap = p.segcap;
     const size_t pitch = 4u * static_cast<size_t>(p.seg_stride);
     const uint32_t trigger = segcap - 32u;  // exact: above it the next tile could overflow
     const uint32_t lt = (1u << lane) - 1u;
     if constexpr (MODE == kModeExact) {
-      for (int i = rank; i < kHistBins; i += 128) sm.cut[g].hist[i] = 0u;  // the selects keep it zero
+      for (int i = rank; i < kHistBins; i += 128) sm.cut[sub].hist[i] = 0u;  // the selects keep it zero
     }
     uint32_t use = 0;
     bool ok = true;
@@ -316,21 +336,21 @@ __global__ void __launch_bounds__(384, 1)
       const int qb = block_of(r);
       if (qb < 0) break;
       const int row_base = qb * C::QB + qbase;
-      for (int e = rank; e < C::QPM * H; e += 128) {
-        const int qi = e / H, j = e % H, row = row_base + qi;
+      for (int i = rank; i < QPW * H; i += 128) {
+        const int qi = i / H, j = i % H, row = row_base + qi;
         sm.wq[qbase + qi][j] = (row < p.Lq) ? __ldg(&p.w[static_cast<size_t>(row) * H + j]) * 0x1p25f
                                             : 0.0f;
       }
-      for (int qi = rank; qi < C::QPM; qi += 128) {
+      for (int qi = rank; qi < QPW; qi += 128) {
         const int row = row_base + qi;
         sm.sq[qbase + qi] = (row < p.Lq) ? __ldg(&p.q_scale[row]) : 0.0f;
         sm.thr[qbase + qi] = (MODE == kModeLean && row < p.Lq) ? __ldcg(p.thr + row) : 0ull;
       }
-      if (rank == 0) sm.cflag[g] = 0u;
+      if (rank == 0) sm.cflag[sub] = 0u;
       gs.sync();
-      uint32_t cw[C::QPM];  // keys in this warp's segment, per query (warp-uniform)
+      uint32_t cw[QPW];  // keys in this warp's segment, per query (warp-uniform)
 #pragma unroll
-      for (int qi = 0; qi < C::QPM; ++qi) cw[qi] = 0u;
+      for (int qi = 0; qi < QPW; ++qi) cw[qi] = 0u;
       const int nt = ntiles_of(qb);
       int v = static_cast<int>(wl * 32u + lane);  // this thread's row of the key tensor map
       auto scale_of = [&](int vi) {
@@ -346,22 +366,24 @@ __global__ void __launch_bounds__(384, 1)
         good = good && got;
         __syncwarp();
         tc_fence_after();
-        float score_part[C::QPM];
+        // This warp's QPW * H columns in chunks of 32.
+        constexpr int NCH = QPW * H / 32;
+        float score_part[QPW];
         uint32_t ra[32], rb[32];
         tmem_ld_32x32b_x32(taddr0, ra);
         tmem_wait_ld_regs(ra);
         if constexpr (H == 64) {
-          // 4 queries x 64 heads: packed FMA over head pairs, four float2 partial sums per query.
-          float2 acc[C::QPM][4];
+          // 64 heads per query: packed FMA over head pairs, four float2 partial sums per query.
+          float2 acc[QPW][4];
 #pragma unroll
-          for (int qi = 0; qi < C::QPM; ++qi)
+          for (int qi = 0; qi < QPW; ++qi)
 #pragma unroll
             for (int a = 0; a < 4; ++a) acc[qi][a] = make_float2(0.0f, 0.0f);
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
+          for (int c = 0; c < NCH; ++c) {
             uint32_t(&cur)[32] = (c & 1) ? rb : ra;
             uint32_t(&nxt)[32] = (c & 1) ? ra : rb;
-            if (c + 1 < 8) tmem_ld_32x32b_x32(taddr0 + (c + 1) * 32, nxt);
+            if (c + 1 < NCH) tmem_ld_32x32b_x32(taddr0 + (c + 1) * 32, nxt);
             const int qi = c >> 1;
 #pragma unroll
             for (int j = 0; j < 32; j += 4) {
@@ -371,25 +393,25 @@ __global__ void __launch_bounds__(384, 1)
               const float r1 = __saturatef(__uint_as_float(cur[j + 1]) * 0x1p-25f);
               const float r2 = __saturatef(__uint_as_float(cur[j + 2]) * 0x1p-25f);
               const float r3 = __saturatef(__uint_as_float(cur[j + 3]) * 0x1p-25f);
-              const int a = ((j >> 2) & 1) * 2;
+              const int a = QPW >= 4 ? ((j >> 2) & 1) * 2 : 0;  // fewer chains when registers are scarce
               acc[qi][a] = __ffma2_rn(make_float2(wv.x, wv.y), make_float2(r0, r1), acc[qi][a]);
               acc[qi][a + 1] = __ffma2_rn(make_float2(wv.z, wv.w), make_float2(r2, r3), acc[qi][a + 1]);
             }
-            if (c + 1 < 8) tmem_wait_ld_regs(nxt);
+            if (c + 1 < NCH) tmem_wait_ld_regs(nxt);
           }
 #pragma unroll
-          for (int qi = 0; qi < C::QPM; ++qi)
+          for (int qi = 0; qi < QPW; ++qi)
             score_part[qi] = ((acc[qi][0].x + acc[qi][0].y) + (acc[qi][1].x + acc[qi][1].y)) +
                              ((acc[qi][2].x + acc[qi][2].y) + (acc[qi][3].x + acc[qi][3].y));
         } else {
-          // 32 queries x 8 heads: one scalar chain per query, four queries per chunk.
+          // 8 heads per query: one scalar chain per query, four queries per chunk.
 #pragma unroll
-          for (int qi = 0; qi < C::QPM; ++qi) score_part[qi] = 0.0f;
+          for (int qi = 0; qi < QPW; ++qi) score_part[qi] = 0.0f;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
+          for (int c = 0; c < NCH; ++c) {
             uint32_t(&cur)[32] = (c & 1) ? rb : ra;
             uint32_t(&nxt)[32] = (c & 1) ? ra : rb;
-            if (c + 1 < 8) tmem_ld_32x32b_x32(taddr0 + (c + 1) * 32, nxt);
+            if (c + 1 < NCH) tmem_ld_32x32b_x32(taddr0 + (c + 1) * 32, nxt);
 #pragma unroll
             for (int j = 0; j < 32; j += 4) {
               const int col = c * 32 + j;
@@ -400,7 +422,7 @@ __global__ void __launch_bounds__(384, 1)
               score_part[qi] = fmaf(wv.z, __saturatef(__uint_as_float(cur[j + 2]) * 0x1p-25f), score_part[qi]);
               score_part[qi] = fmaf(wv.w, __saturatef(__uint_as_float(cur[j + 3]) * 0x1p-25f), score_part[qi]);
             }
-            if (c + 1 < 8) tmem_wait_ld_regs(nxt);
+            if (c + 1 < NCH) tmem_wait_ld_regs(nxt);
           }
         }
         tc_fence_before();
@@ -411,7 +433,7 @@ __global__ void __launch_bounds__(384, 1)
         // Appends to this warp's own segment: no atomics, the count lives in a register.
         uint32_t flags = 0u;
 #pragma unroll
-        for (int qi = 0; qi < C::QPM; ++qi) {
+        for (int qi = 0; qi < QPW; ++qi) {
           const int row = row_base + qi;
           const bool valid = (row < p.Lq) && (v < p.nkeys) && (s <= p.q_pos0 + row);
           const float score = (score_part[qi] * sm.sq[qbase + qi]) * sk;
@@ -424,41 +446,41 @@ __global__ void __launch_bounds__(384, 1)
           if constexpr (MODE == kModeExact) flags |= (cw[qi] > trigger) ? (1u << qi) : 0u;
         }
         if constexpr (MODE == kModeExact) {
-          // Cut-backs: one decision for the whole warpgroup. The barrier ORs the warps'
-          // requests, and the flag word written before it is visible to every warp after it.
-          if (flags && lane == 0) atomicOr(&sm.cflag[g], flags);
-          if (named_bar_or(1u + g, 128, flags != 0u)) {
-            const uint32_t mask = *reinterpret_cast<volatile uint32_t*>(&sm.cflag[g]);
+          // Cut-backs: one decision for the whole group. The barrier ORs the warps' requests,
+          // and the flag word written before it is visible to every warp after it.
+          if (flags && lane == 0) atomicOr(&sm.cflag[sub], flags);
+          if (named_bar_or(1u + sub, 128, flags != 0u)) {
+            const uint32_t mask = *reinterpret_cast<volatile uint32_t*>(&sm.cflag[sub]);
             if (lane == 0) {
 #pragma unroll
-              for (int qi = 0; qi < C::QPM; ++qi) sm.wcnt[qbase + qi][wl] = cw[qi];
+              for (int qi = 0; qi < QPW; ++qi) sm.wcnt[qbase + qi][wl] = cw[qi];
             }
             gs.sync();
-            if (rank == 0) sm.cflag[g] = 0u;
+            if (rank == 0) sm.cflag[sub] = 0u;
 #pragma unroll 1
-            for (int qi = 0; qi < C::QPM; ++qi) {
+            for (int qi = 0; qi < QPW; ++qi) {
               if ((mask >> qi) & 1u)
                 cut_back(p.cand + static_cast<size_t>(row_base + qi) * pitch, p.seg_stride,
-                         sm.wcnt[qbase + qi], &sm.thr[qbase + qi], &sm.cut[g], k, rank, 1u + g);
+                         sm.wcnt[qbase + qi], &sm.thr[qbase + qi], &sm.cut[sub], k, rank, 1u + sub);
             }
 #pragma unroll
-            for (int qi = 0; qi < C::QPM; ++qi) cw[qi] = sm.wcnt[qbase + qi][wl];
+            for (int qi = 0; qi < QPW; ++qi) cw[qi] = sm.wcnt[qbase + qi][wl];
           }
         }
       }
-      ok = named_bar_and(1u + g, 128, ok && good);
+      ok = named_bar_and(1u + sub, 128, ok && good);
       if (!ok) break;
-      // Segment counts (and thresholds) of every query of this warpgroup.
+      // Segment counts (and thresholds) of every query of this group.
       if (lane == 0) {
 #pragma unroll
-        for (int qi = 0; qi < C::QPM; ++qi) {
+        for (int qi = 0; qi < QPW; ++qi) {
           const int row = row_base + qi;
           if (row < p.Lq) p.counts[static_cast<size_t>(row) * 4 + wl] = cw[qi];
           sm.wcnt[qbase + qi][wl] = cw[qi];
         }
       }
       if constexpr (MODE == kModeExact) {
-        for (int qi = rank; qi < C::QPM; qi += 128) {
+        for (int qi = rank; qi < QPW; qi += 128) {
           const int row = row_base + qi;
           if (row < p.Lq) p.thr[row] = sm.thr[qbase + qi];
         }
@@ -468,7 +490,7 @@ __global__ void __launch_bounds__(384, 1)
         // appended), or whose segment overflowed, sends its block to the exact mode.
         gs.sync();
         bool bad = false;
-        for (int qi = rank; qi < C::QPM; qi += 128) {
+        for (int qi = rank; qi < QPW; qi += 128) {
           const int row = row_base + qi;
           if (row >= p.Lq) continue;
           uint32_t total = 0;
@@ -517,7 +539,7 @@ static dsa_status launch_mode(const CUtensorMap& tq, const CUtensorMap& tk, cons
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return DSA_ERR_CUDA;
-  kern<<<grid, C::THREADS, smem, stream>>>(tq, tk, p);
+  kern<<<grid, PRoles<H, MODE>::THREADS, smem, stream>>>(tq, tk, p);
   return cuda_status(cudaGetLastError());
 }
 
