@@ -97,7 +97,8 @@ dsa_status launch_prefill_finish(const uint64_t* cand, const uint32_t* counts,
 // Per prefill row, the threshold of the lean pass from the row's sampled keys.
 dsa_status launch_prefill_sample_threshold(const uint64_t* cand, const uint32_t* counts,
                                            uint64_t* thr, uint32_t seg_stride, int rows,
-                                           int q_pos0, int Lk, int topk, cudaStream_t stream);
+                                           int q_pos0, int Lk, int topk, uint32_t max_samples,
+                                           cudaStream_t stream);
 dsa_status launch_decode(const DecodeLaunch& a);
 dsa_status launch_decode_topk(const float* scores, int max_len, const int32_t* seq_lens,
                               const uint32_t* bins, int B, int topk, int32_t* out_idx,

@@ -590,7 +590,7 @@ static dsa_status launch_prefill_t(const PrefillLaunch& a) {
     ps.segcap = L.seg_stride;
     if ((st = launch_mode<H, D, kModeSample>(tq, ts, ps, grid, a.stream)) != DSA_OK) return st;
     if ((st = launch_prefill_sample_threshold(p.cand, p.counts, p.thr, L.seg_stride, a.Lq, a.q_pos0,
-                                              a.Lk, a.topk, a.stream)) != DSA_OK)
+                                              a.Lk, a.topk, static_cast<uint32_t>(nks), a.stream)) != DSA_OK)
       return st;
     // Lean pass with those thresholds; blocks it cannot finish are listed for the exact mode.
     if (cudaMemsetAsync(base + L.flags_off, 0, L.total - L.flags_off, a.stream) != cudaSuccess)

@@ -246,12 +246,14 @@ dsa_status launch_prefill_finish(const uint64_t* cand, const uint32_t* counts,
 // the k-th largest key is a 6.5-sigma event, and otherwise at least k keys of the row are >= T.
 // A row with r >= n_s (short rows, n <= k) gets T = 0: every key is kept. (The lean pass checks
 // the count it actually appended and hands the rare failure to the exact pass.)
-constexpr int kSampleThreads = 128;
+constexpr int kSampleThreads = 256;
 
 __global__ void __launch_bounds__(kSampleThreads)
     prefill_sample_threshold_kernel(const uint64_t* __restrict__ cand, const uint32_t* __restrict__ counts,
                                     uint64_t* __restrict__ thr, uint32_t seg_stride, int q_pos0, int Lk,
-                                    int topk) {
+                                    int topk, uint32_t stage_cap) {
+  extern __shared__ uint8_t smem_raw[];
+  uint64_t* stage = reinterpret_cast<uint64_t*>(smem_raw);  // stage_cap keys
   __shared__ uint32_t hist[kHistBins];
   __shared__ GroupScratch<kSampleThreads> sc;
   const GroupSync<kSampleThreads> gs{0};
@@ -273,22 +275,50 @@ __global__ void __launch_bounds__(kSampleThreads)
     return;
   }
   const uint32_t r = static_cast<uint32_t>(ceil(rr));
-  for (uint32_t b = rank; b < kHistBins; b += kSampleThreads) hist[b] = 0u;
-  gs.sync();
-  auto key_at = [&](uint32_t e) {
+  auto src_at = [&](uint32_t e) {
     const uint32_t w = (e >= o1 ? 1u : 0u) + (e >= o2 ? 1u : 0u) + (e >= o3 ? 1u : 0u);
     const uint32_t start = e >= o3 ? o3 : (e >= o2 ? o2 : (e >= o1 ? o1 : 0u));
     return __ldcg(buf + w * seg_stride + (e - start));
   };
-  const uint64_t T = group_kth_threshold<kSampleThreads>(key_at, ns, r, rank, hist, sc, gs);
+  for (uint32_t b = rank; b < kHistBins; b += kSampleThreads) hist[b] = 0u;
+  uint64_t T;
+  if (ns <= stage_cap) {
+    // Stage the samples in shared memory (eight loads in flight per thread), select there.
+    for (uint32_t e0 = 0; e0 < ns; e0 += 8 * kSampleThreads) {
+      uint64_t v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t e = e0 + i * kSampleThreads + rank;
+        v[i] = e < ns ? src_at(e) : 0ull;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t e = e0 + i * kSampleThreads + rank;
+        if (e < ns) stage[e] = v[i];
+      }
+    }
+    gs.sync();
+    T = group_kth_threshold<kSampleThreads>([&](uint32_t e) { return stage[e]; }, ns, r, rank, hist, sc, gs);
+  } else {
+    gs.sync();
+    T = group_kth_threshold<kSampleThreads>(src_at, ns, r, rank, hist, sc, gs);
+  }
   if (rank == 0) thr[row] = T;
 }
 
 dsa_status launch_prefill_sample_threshold(const uint64_t* cand, const uint32_t* counts,
                                            uint64_t* thr, uint32_t seg_stride, int rows,
-                                           int q_pos0, int Lk, int topk, cudaStream_t stream) {
-  prefill_sample_threshold_kernel<<<rows, kSampleThreads, 0, stream>>>(cand, counts, thr, seg_stride,
-                                                                       q_pos0, Lk, topk);
+                                           int q_pos0, int Lk, int topk, uint32_t max_samples,
+                                           cudaStream_t stream) {
+  // Shared staging for up to max_samples keys (at most 64 KB; longer samples select from global).
+  const uint32_t stage_cap = max_samples < 8192u ? max_samples : 8192u;
+  const size_t smem = static_cast<size_t>(stage_cap) * sizeof(uint64_t);
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(prefill_sample_threshold_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  prefill_sample_threshold_kernel<<<rows, kSampleThreads, smem, stream>>>(cand, counts, thr, seg_stride,
+                                                                          q_pos0, Lk, topk, stage_cap);
   return cuda_status(cudaGetLastError());
 }
 
