@@ -26,7 +26,7 @@ struct DCfg {
   static constexpr int PAGE = 64;              // keys per cache block
   static constexpr int BN = 128;               // keys per tile
   static constexpr int STAGES = 3;
-  static constexpr int TPC = 8;                // tiles per CTA
+  static constexpr int TPC = 16;               // tiles per CTA
   static constexpr int QTILE = H * D;
   static constexpr int KTILE = BN * D;
   static constexpr int PAGE_BYTES = PAGE * D;

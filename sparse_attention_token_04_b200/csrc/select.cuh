@@ -397,3 +397,94 @@ __device__ uint64_t* group_merge_sort_desc(Load load, uint64_t* a, uint64_t* b, 
 }
 
 }  // namespace dsa
+
+namespace dsa {
+
+// Ranks the m distinct keys tmp[0..m) (m <= KPT * NT) by a bucket sort and leaves the
+// min(m, k) largest in tmp[0..min(m, k)) in descending order. NBK buckets of equal width in
+// score value span [score(omin), score(omax)] (omin / omax: order-preserving score bits of the
+// smallest and largest key); the fp32 map from score to bucket is monotone, so a larger key
+// never lands in a lower bucket. A suffix scan gives each bucket's first rank, the buckets'
+// keys are placed side by side, and a key's rank is its bucket's first rank plus the number
+// of larger keys in its bucket. bk (NBK words) must be zero on entry. Returns false, with bk
+// zero again and tmp unchanged, when some bucket holds more than max_bucket keys (heavy ties,
+// scores bunched in a sliver of the span): the caller then sorts another way.
+template <int NT, int KPT, int NBK>
+__device__ bool group_bucket_rank(uint64_t* tmp, uint32_t m, uint32_t k, uint32_t omin, uint32_t omax,
+                                  uint32_t max_bucket, uint32_t* bk, uint32_t* flag,
+                                  GroupScratch<NT>& sc, const GroupSync<NT>& gs, uint32_t rank) {
+  static_assert(NBK % NT == 0, "buckets per thread");
+  const float smin = ordered_to_float(omin), smax = ordered_to_float(omax);
+  const float span = smax - smin;
+  // A zero (or overflowing) span puts every key in bucket 0.
+  const float scale = (span > 0.0f && span < 3.0e38f) ? (NBK - 0.5f) / span : 0.0f;
+  if (rank == 0) *flag = 0u;
+  gs.sync();
+  uint64_t v[KPT];
+  uint32_t bs[KPT];  // bucket << 16 | slot in the bucket; later the key's rank
+#pragma unroll
+  for (int i = 0; i < KPT; ++i) {
+    const uint32_t e = rank + i * NT;
+    v[i] = 0ull;
+    bs[i] = 0u;
+    if (e < m) {
+      v[i] = tmp[e];
+      const float f = (key_score(v[i]) - smin) * scale;
+      const uint32_t b = min(static_cast<uint32_t>(f > 0.0f ? f : 0.0f), static_cast<uint32_t>(NBK - 1));
+      const uint32_t slot = atomicAdd(&bk[b], 1u);
+      bs[i] = (b << 16) | slot;
+      if (slot >= max_bucket) *flag = 1u;
+    }
+  }
+  gs.sync();
+  if (*flag) {
+    for (uint32_t b = rank; b < static_cast<uint32_t>(NBK); b += NT) bk[b] = 0u;
+    gs.sync();
+    return false;
+  }
+  // First rank of each bucket: keys in higher buckets (exclusive suffix sum), in place.
+  constexpr int BPT = NBK / NT;
+  uint32_t cnt[BPT];
+  uint32_t local = 0;
+#pragma unroll
+  for (int i = 0; i < BPT; ++i) {
+    cnt[i] = bk[rank * BPT + i];
+    local += cnt[i];
+  }
+  uint32_t acc = group_suffix_exclusive<NT>(local, rank, sc.w, gs, nullptr);
+#pragma unroll
+  for (int i = BPT - 1; i >= 0; --i) {
+    bk[rank * BPT + i] = acc;
+    acc += cnt[i];
+  }
+  gs.sync();
+  // Bucket members side by side (every key is in registers by now).
+#pragma unroll
+  for (int i = 0; i < KPT; ++i) {
+    const uint32_t e = rank + i * NT;
+    if (e < m) tmp[bk[bs[i] >> 16] + (bs[i] & 0xFFFFu)] = v[i];
+  }
+  gs.sync();
+#pragma unroll
+  for (int i = 0; i < KPT; ++i) {
+    const uint32_t e = rank + i * NT;
+    if (e < m) {
+      const uint32_t b = bs[i] >> 16;
+      const uint32_t s0 = bk[b];
+      const uint32_t nb = (b == 0 ? m : bk[b - 1]) - s0;
+      uint32_t r = s0;
+      for (uint32_t j = 0; j < nb; ++j) r += tmp[s0 + j] > v[i] ? 1u : 0u;
+      bs[i] = r;
+    }
+  }
+  gs.sync();
+#pragma unroll
+  for (int i = 0; i < KPT; ++i) {
+    const uint32_t e = rank + i * NT;
+    if (e < m && bs[i] < k) tmp[bs[i]] = v[i];
+  }
+  gs.sync();
+  return true;
+}
+
+}  // namespace dsa

@@ -9,8 +9,8 @@
 //                           kernel has already counted the request's scores in 2048 bins of
 //                           their order-preserving top 11 bits; the bin holding the k-th score
 //                           bounds the candidates, which one pass over the scores collects into
-//                           shared memory. An exact radix select there and a merge sort finish
-//                           the row, in the same order and padding.
+//                           shared memory. The bucket ranking of the finish kernel orders them
+//                           (radix select + merge sort with heavy ties), same order and padding.
 #include "common.cuh"
 #include "internal.h"
 #include "select.cuh"
@@ -122,77 +122,11 @@ __global__ void __launch_bounds__(kFinishThreads)
   bool need_select = m > kFinishTmp;
   auto tmp_at = [&](uint32_t i) { return sm.tmp[i]; };
   if (!need_select && m > 0) {
-    const float smin = ordered_to_float(sm.omin), smax = ordered_to_float(sm.omax);
-    const float span = smax - smin;
-    // Buckets of equal width in score; a zero (or overflowing) span puts every key in bucket 0.
-    const float scale = (span > 0.0f && span < 3.0e38f) ? (kFinishBuckets - 0.5f) / span : 0.0f;
-    uint64_t v[kFinishKPT];
-    uint32_t bs[kFinishKPT];  // bucket << 16 | slot in the bucket
-#pragma unroll
-    for (int i = 0; i < kFinishKPT; ++i) {
-      const uint32_t e = rank + i * kFinishThreads;
-      v[i] = 0ull;
-      bs[i] = 0u;
-      if (e < m) {
-        v[i] = sm.tmp[e];
-        const float f = (key_score(v[i]) - smin) * scale;
-        const uint32_t b = min(static_cast<uint32_t>(f > 0.0f ? f : 0.0f), static_cast<uint32_t>(kFinishBuckets - 1));
-        const uint32_t slot = atomicAdd(&sm.bk[b], 1u);
-        bs[i] = (b << 16) | slot;
-        if (slot >= kBucketMax) sm.big = 1u;
-      }
-    }
-    gs.sync();
-    if (sm.big) {
-      need_select = true;
-      for (uint32_t b = rank; b < kFinishBuckets; b += kFinishThreads) sm.bk[b] = 0u;
-      gs.sync();
-    } else {
-      // First rank of each bucket: keys in higher buckets (exclusive suffix sum), in place.
-      constexpr int BPT = kFinishBuckets / kFinishThreads;
-      uint32_t cnt[BPT];
-      uint32_t local = 0;
-#pragma unroll
-      for (int i = 0; i < BPT; ++i) {
-        cnt[i] = sm.bk[rank * BPT + i];
-        local += cnt[i];
-      }
-      uint32_t acc = group_suffix_exclusive<kFinishThreads>(local, rank, sm.sc.w, gs, nullptr);
-#pragma unroll
-      for (int i = BPT - 1; i >= 0; --i) {
-        sm.bk[rank * BPT + i] = acc;
-        acc += cnt[i];
-      }
-      gs.sync();
-      // Bucket members side by side (every key is in registers by now).
-#pragma unroll
-      for (int i = 0; i < kFinishKPT; ++i) {
-        const uint32_t e = rank + i * kFinishThreads;
-        if (e < m) sm.tmp[sm.bk[bs[i] >> 16] + (bs[i] & 0xFFFFu)] = v[i];
-      }
-      gs.sync();
-      // Rank = first rank of the bucket + members of the bucket that are larger.
-#pragma unroll
-      for (int i = 0; i < kFinishKPT; ++i) {
-        const uint32_t e = rank + i * kFinishThreads;
-        if (e < m) {
-          const uint32_t b = bs[i] >> 16;
-          const uint32_t s0 = sm.bk[b];
-          const uint32_t nb = (b == 0 ? m : sm.bk[b - 1]) - s0;
-          uint32_t r = s0;
-          for (uint32_t j = 0; j < nb; ++j) r += sm.tmp[s0 + j] > v[i] ? 1u : 0u;
-          bs[i] = r;
-        }
-      }
-      gs.sync();
-#pragma unroll
-      for (int i = 0; i < kFinishKPT; ++i) {
-        const uint32_t e = rank + i * kFinishThreads;
-        if (e < m && bs[i] < k) sm.tmp[bs[i]] = v[i];
-      }
-      gs.sync();
+    if (group_bucket_rank<kFinishThreads, kFinishKPT, kFinishBuckets>(
+            sm.tmp, m, k, sm.omin, sm.omax, kBucketMax, sm.bk, &sm.big, sm.sc, gs, rank))
       n_res = m < k ? m : k;
-    }
+    else
+      need_select = true;
   }
   if (need_select) {
     // Exact radix select of the k-th key and a merge sort of the winners. bk is zero here.
@@ -324,16 +258,18 @@ dsa_status launch_prefill_sample_threshold(const uint64_t* cand, const uint32_t*
 
 constexpr int kDecodeTopkThreads = 1024;
 constexpr uint32_t kDecodeCandCap = 8192;
+constexpr int kDecodeBuckets = 4096;
 
 struct DecodeTopkSmem {
-  uint64_t a[kSortBuf];             // sort buffer
-  uint64_t win[DSA_MAX_TOPK];       // the k winners, contiguous
-  uint64_t cand[kDecodeCandCap];    // candidates; later the second sort buffer
+  uint64_t a[kSortBuf];             // sort buffer; before that the bucket counts of the ranking
+  uint64_t win[DSA_MAX_TOPK];       // the k winners, contiguous (select path)
+  uint64_t cand[kDecodeCandCap];    // candidates, ranked in place; or the second sort buffer
   uint32_t hist[kHistBins];
   GroupScratch<kDecodeTopkThreads> sc;
-  uint32_t n_cand;
+  uint32_t n_cand, big, omin, omax;
 };
 static_assert(kDecodeCandCap >= static_cast<uint32_t>(kSortBuf), "second sort buffer");
+static_assert(sizeof(uint64_t) * kSortBuf >= sizeof(uint32_t) * kDecodeBuckets, "bucket counts in a");
 
 __global__ void __launch_bounds__(kDecodeTopkThreads)
     decode_topk_kernel(const float* __restrict__ scores, int max_len,
@@ -354,14 +290,20 @@ __global__ void __launch_bounds__(kDecodeTopkThreads)
   const float* row = scores + static_cast<size_t>(req) * max_len;
   auto key_at = [&](uint32_t e) { return make_key(__ldcg(row + e), e); };
   const uint32_t un = static_cast<uint32_t>(n), k = static_cast<uint32_t>(topk);
-  const uint32_t P = sort_size(k);
-  uint32_t n_win = un < k ? un : k;
+  uint32_t* bk = reinterpret_cast<uint32_t*>(sm.a);
+  for (uint32_t b = rank; b < static_cast<uint32_t>(kDecodeBuckets); b += kDecodeTopkThreads) bk[b] = 0u;
+  if (rank == 0) {
+    sm.n_cand = 0u;
+    sm.omin = 0xFFFFFFFFu;
+    sm.omax = 0u;
+  }
 
+  // Boundary bin: the highest bin where the count of scores at or above it reaches k (bin 0
+  // when the request has at most k keys: every key is a winner).
+  uint32_t bstar = 0, n_cand = un;
   if (un > k) {
-    // Boundary bin: the highest bin where the count of scores at or above it reaches k.
     for (uint32_t b = rank; b < kHistBins; b += kDecodeTopkThreads)
       sm.hist[b] = bins[static_cast<size_t>(req) * kHistBins + b];
-    if (rank == 0) sm.n_cand = 0;
     gs.sync();
     constexpr int BPT = kHistBins / kDecodeTopkThreads;
     uint32_t local = 0;
@@ -378,59 +320,89 @@ __global__ void __launch_bounds__(kDecodeTopkThreads)
       acc += c;
     }
     gs.sync();
-    const uint32_t bstar = sm.sc.w[kDecodeTopkThreads / 32];
-    const uint32_t n_cand = sm.sc.w[kDecodeTopkThreads / 32 + 1];
+    bstar = sm.sc.w[kDecodeTopkThreads / 32];
+    n_cand = sm.sc.w[kDecodeTopkThreads / 32 + 1];
     gs.sync();
-    for (uint32_t b = rank; b < kHistBins; b += kDecodeTopkThreads) sm.hist[b] = 0u;  // selects below need it zero
-    gs.sync();
-    uint64_t T;
-    if (n_cand <= kDecodeCandCap) {
-      // One pass: keys whose bin is at or above the boundary bin, eight loads in flight.
-      for (uint32_t e0 = 0; e0 < un; e0 += 8 * kDecodeTopkThreads) {
-        uint64_t v[8];
+  }
+  for (uint32_t b = rank; b < kHistBins; b += kDecodeTopkThreads) sm.hist[b] = 0u;  // selects below need it zero
+  gs.sync();
+
+  const uint64_t* res = sm.cand;
+  bool padded = false;
+  uint32_t n_res = 0;
+  if (n_cand <= kDecodeCandCap) {
+    // One pass: keys whose bin is at or above the boundary bin, 32 score loads in flight per
+    // thread (a 200000-key request in seven rounds), with their score range.
+    constexpr int kInFlight = 32;
+    uint32_t lmin = 0xFFFFFFFFu, lmax = 0u;
+    for (uint32_t e0 = 0; e0 < un; e0 += kInFlight * kDecodeTopkThreads) {
+      float v[kInFlight];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint32_t e = e0 + i * kDecodeTopkThreads + rank;
-          v[i] = e < un ? key_at(e) : 0ull;
-        }
+      for (int i = 0; i < kInFlight; ++i) {
+        const uint32_t e = e0 + i * kDecodeTopkThreads + rank;
+        v[i] = e < un ? __ldcg(row + e) : 0.0f;
+      }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const bool take = v[i] != 0ull && static_cast<uint32_t>(v[i] >> 53) >= bstar;
-          const uint32_t m = __ballot_sync(0xFFFFFFFFu, take);
-          if (m) {
-            uint32_t base = 0;
-            if (lane == 0) base = atomicAdd(&sm.n_cand, static_cast<uint32_t>(__popc(m)));
-            base = __shfl_sync(0xFFFFFFFFu, base, 0);
-            const uint32_t pos = base + __popc(m & ((1u << lane) - 1u));
-            if (take && pos < kDecodeCandCap) sm.cand[pos] = v[i];
+      for (int i = 0; i < kInFlight; ++i) {
+        const uint32_t e = e0 + i * kDecodeTopkThreads + rank;
+        const uint64_t key = make_key(v[i], e);
+        const bool take = e < un && static_cast<uint32_t>(key >> 53) >= bstar;
+        const uint32_t m = __ballot_sync(0xFFFFFFFFu, take);
+        if (m) {
+          uint32_t base = 0;
+          if (lane == 0) base = atomicAdd(&sm.n_cand, static_cast<uint32_t>(__popc(m)));
+          base = __shfl_sync(0xFFFFFFFFu, base, 0);
+          const uint32_t pos = base + __popc(m & ((1u << lane) - 1u));
+          if (take && pos < kDecodeCandCap) sm.cand[pos] = key;
+          if (take) {
+            const uint32_t o = static_cast<uint32_t>(key >> 32);
+            lmin = o < lmin ? o : lmin;
+            lmax = o > lmax ? o : lmax;
           }
         }
       }
-      gs.sync();
-      const uint32_t got = sm.n_cand < kDecodeCandCap ? sm.n_cand : kDecodeCandCap;
-      if (got != n_cand && rank == 0) record_error(hdr, DSA_ERR_DEVICE, DETAIL_HIST_MISMATCH);
+    }
+    lmin = __reduce_min_sync(0xFFFFFFFFu, lmin);
+    lmax = __reduce_max_sync(0xFFFFFFFFu, lmax);
+    if (lane == 0 && lmax != 0u) {
+      atomicMin(&sm.omin, lmin);
+      atomicMax(&sm.omax, lmax);
+    }
+    gs.sync();
+    const uint32_t got = sm.n_cand < kDecodeCandCap ? sm.n_cand : kDecodeCandCap;
+    if (got != n_cand && rank == 0) record_error(hdr, DSA_ERR_DEVICE, DETAIL_HIST_MISMATCH);
+    if (got > 0 &&
+        group_bucket_rank<kDecodeTopkThreads, kDecodeCandCap / kDecodeTopkThreads, kDecodeBuckets>(
+            sm.cand, got, k, sm.omin, sm.omax, 256u, bk, &sm.big, sm.sc, gs, rank)) {
+      n_res = got < k ? got : k;
+    } else {
+      // Heavy ties: exact radix select over the candidates, then a merge sort.
       auto cand_at = [&](uint32_t e) { return sm.cand[e]; };
-      T = got > k ? group_kth_threshold<kDecodeTopkThreads>(cand_at, got, k, rank, sm.hist, sm.sc, gs)
-                  : 0ull;
-      n_win = group_compact_ge<kDecodeTopkThreads>(
+      const uint64_t T = got > k ? group_kth_threshold<kDecodeTopkThreads>(cand_at, got, k, rank, sm.hist, sm.sc, gs)
+                                 : 0ull;
+      uint32_t nw = group_compact_ge<kDecodeTopkThreads>(
           cand_at, got, T, [&](uint32_t pos, uint64_t key) { if (pos < k) sm.win[pos] = key; }, rank,
           sm.sc, gs);
-    } else {
-      // Too many keys share the boundary bin (heavy ties): radix select over global memory.
-      T = group_kth_threshold<kDecodeTopkThreads>(key_at, un, k, rank, sm.hist, sm.sc, gs);
-      n_win = group_compact_ge<kDecodeTopkThreads>(
-          key_at, un, T, [&](uint32_t pos, uint64_t key) { if (pos < k) sm.win[pos] = key; }, rank,
-          sm.sc, gs);
+      nw = nw < k ? nw : k;
+      res = group_merge_sort_desc<kDecodeTopkThreads>(
+          [&](uint32_t e) { return e < nw ? sm.win[e] : 0ull; }, sm.a, sm.cand, sort_size(k), rank, gs);
+      padded = true;
+      n_res = nw;
     }
-    n_win = n_win < k ? n_win : k;
   } else {
-    for (uint32_t e = rank; e < un; e += kDecodeTopkThreads) sm.win[e] = key_at(e);
+    // Too many keys share the boundary bin (heavy ties): radix select over global memory.
+    const uint64_t T = group_kth_threshold<kDecodeTopkThreads>(key_at, un, k, rank, sm.hist, sm.sc, gs);
+    uint32_t nw = group_compact_ge<kDecodeTopkThreads>(
+        key_at, un, T, [&](uint32_t pos, uint64_t key) { if (pos < k) sm.win[pos] = key; }, rank,
+        sm.sc, gs);
+    nw = nw < k ? nw : k;
+    res = group_merge_sort_desc<kDecodeTopkThreads>(
+        [&](uint32_t e) { return e < nw ? sm.win[e] : 0ull; }, sm.a, sm.cand, sort_size(k), rank, gs);
+    padded = true;
+    n_res = nw;
   }
-  gs.sync();
-  const uint64_t* s = group_merge_sort_desc<kDecodeTopkThreads>(
-      [&](uint32_t e) { return e < n_win ? sm.win[e] : 0ull; }, sm.a, sm.cand, P, rank, gs);
   for (uint32_t e = rank; e < k; e += kDecodeTopkThreads) {
-    const uint64_t key = s[spad(e)];
+    const uint64_t key = e < n_res ? res[padded ? spad(e) : e] : 0ull;
     out_idx[static_cast<size_t>(req) * topk + e] = key_index(key);
     if (out_score) out_score[static_cast<size_t>(req) * topk + e] = key_score(key);
   }
