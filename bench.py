@@ -527,6 +527,68 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def run_long_prefill_patterns(args, local):
+    """Long-context prefill under several IndexCache patterns: L = 200000, H = 64, d = 128,
+    k = 2048, 47 rho = 0.9 correlated layers, chunks of 8192 queries against the whole causal
+    prefix. Every layer's indexer pass (all 25 chunks) is timed once with CUDA events; an F/S
+    pattern runs exactly its F layers (S layers alias their F buffer: no launch), so its wall
+    time is the sum over its F layers. Prints one JSON line."""
+    from sparse_attention_token_04_b200 import binding as B
+    from synth import SEARCHED_QUARTER_PATTERN, correlated_layers
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    L, H, d, topk, n_layers, chunk = 200000, 64, 128, 2048, 47, 8192
+    patterns = {
+        "searched 1/4 (12 F)": SEARCHED_QUARTER_PATTERN,
+        "all F (47 F)": "F" * n_layers,
+        "FFFS (36 F)": ("FFFS" * 12)[:n_layers],
+        "FSSS (12 F)": ("FSSS" * 12)[:n_layers],
+    }
+    ws = torch.empty(B.dsa_prefill_workspace_bytes(chunk, H, d, topk), dtype=torch.uint8, device=device)
+    B.dsa_workspace_init(ws)
+    out_idx = torch.empty(chunk, topk, dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream()
+    layer_ms = []
+    for layer in correlated_layers(L, H, d, n_layers, seed=5, device=device):
+        def one_pass():
+            for c0 in range(0, L, chunk):
+                c1 = min(L, c0 + chunk)
+                B.dsa_indexer_prefill(layer.q[c0:c1], layer.q_scale[c0:c1], layer.w[c0:c1],
+                                      layer.k[:c1], layer.k_scale[:c1], topk, q_pos0=c0,
+                                      out_idx=out_idx[: c1 - c0], want_score=False, workspace=ws)
+        if not layer_ms:
+            one_pass()  # warm-up
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        one_pass()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        layer_ms.append(e0.elapsed_time(e1))
+    status = B.dsa_read_device_status(ws)
+    pairs = causal_pairs(L)
+    flops = 2.0 * H * d * pairs
+    peaks, _ = measured_peaks()
+    fp8_peak = FP8_PER_BF16 * float(peaks["bf16_tflops_sustained"])
+    res = {}
+    for name, pat in patterns.items():
+        f_layers = [i for i, c in enumerate(pat) if c == "F"]
+        ms = float(sum(layer_ms[i] for i in f_layers))
+        res[name] = {"f_layers": len(f_layers), "ms": ms,
+                     "speedup_vs_all_f": float(sum(layer_ms)) / ms}
+    mean_ms = float(np.mean(layer_ms))
+    line = {"workload": "long-context prefill: L=200000, H=64, d=128, k=2048, 47 rho=0.9 "
+                        "correlated FP8 layers, chunks of 8192 queries", "device_status": list(status),
+            "per_layer_ms": {"mean": mean_ms, "min": float(min(layer_ms)), "max": float(max(layer_ms))},
+            "per_layer_pairs_per_s": pairs / (mean_ms / 1e3),
+            "per_layer_tflops": flops / (mean_ms / 1e3) / 1e12,
+            "per_layer_frac_fp8": flops / (mean_ms / 1e3) / 1e12 / fp8_peak,
+            "patterns": res}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -537,6 +599,8 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=50)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-rows", type=int, default=8)
+    ap.add_argument("--long-prefill-patterns", action="store_true",
+                    help="time the 200000-token, 47-layer prefill under four F/S patterns instead")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("at least 3 warm-up steps")
@@ -546,6 +610,9 @@ def main():
             raise SystemExit("launch N > 1 with torch.distributed.run (one process per GPU)")
     if args.impl == "reference":
         run_reference(args, world, rank)
+        return
+    if args.long_prefill_patterns:
+        run_long_prefill_patterns(args, local)
         return
     try:
         run_ours(args, world, rank, local)

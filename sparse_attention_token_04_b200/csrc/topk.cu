@@ -247,8 +247,8 @@ dsa_status launch_prefill_sample_threshold(const uint64_t* cand, const uint32_t*
   // Shared staging for up to max_samples keys (at most 64 KB; longer samples select from global).
   const uint32_t stage_cap = max_samples < 8192u ? max_samples : 8192u;
   const size_t smem = static_cast<size_t>(stage_cap) * sizeof(uint64_t);
-  if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(prefill_sample_threshold_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  // The limit covers the dynamic part only; with the static histogram on top it can pass 48 KB.
+  if (cudaFuncSetAttribute(prefill_sample_threshold_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return DSA_ERR_CUDA;
   prefill_sample_threshold_kernel<<<rows, kSampleThreads, smem, stream>>>(cand, counts, thr, seg_stride,
