@@ -93,7 +93,8 @@ dsa_status launch_prefill(const PrefillLaunch& a);
 // Exact top-k of every row's candidate buffer, ordered and written to out_idx / out_score.
 dsa_status launch_prefill_finish(const uint64_t* cand, const uint32_t* counts,
                                  const uint64_t* thr, uint32_t pitch, int rows, int topk,
-                                 int32_t* out_idx, float* out_score, cudaStream_t stream);
+                                 int32_t* out_idx, float* out_score, int num_sms,
+                                 cudaStream_t stream);
 // Per prefill row, the threshold of the lean pass from the row's sampled keys.
 dsa_status launch_prefill_sample_threshold(const uint64_t* cand, const uint32_t* counts,
                                            uint64_t* thr, uint32_t seg_stride, int rows,

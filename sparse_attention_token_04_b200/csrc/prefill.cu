@@ -605,7 +605,7 @@ static dsa_status launch_prefill_t(const PrefillLaunch& a) {
     if ((st = launch_mode<H, D, kModeExact>(tq, tk, pe, grid, a.stream)) != DSA_OK) return st;
   }
   return launch_prefill_finish(p.cand, p.counts, p.thr, 4u * L.seg_stride, a.Lq, a.topk,
-                               a.out_idx, a.out_score, a.stream);
+                               a.out_idx, a.out_score, a.num_sms, a.stream);
 }
 
 size_t prefill_workspace_bytes(int Lq, int H, int d, int topk, int num_sms) {

@@ -421,7 +421,8 @@ __device__ bool group_bucket_rank(uint64_t* tmp, uint32_t m, uint32_t k, uint32_
   if (rank == 0) *flag = 0u;
   gs.sync();
   uint64_t v[KPT];
-  uint32_t bs[KPT];  // bucket << 16 | slot in the bucket; later the key's rank
+  uint32_t bs[KPT];  // bucket << 16 | slot in the bucket; later the key's rank (~0: no winner)
+  uint32_t bs_bucket[KPT];
 #pragma unroll
   for (int i = 0; i < KPT; ++i) {
     const uint32_t e = rank + i * NT;
@@ -435,6 +436,7 @@ __device__ bool group_bucket_rank(uint64_t* tmp, uint32_t m, uint32_t k, uint32_
       bs[i] = (b << 16) | slot;
       if (slot >= max_bucket) *flag = 1u;
     }
+    bs_bucket[i] = bs[i] >> 16;
   }
   gs.sync();
   if (*flag) {
@@ -458,23 +460,30 @@ __device__ bool group_bucket_rank(uint64_t* tmp, uint32_t m, uint32_t k, uint32_
     acc += cnt[i];
   }
   gs.sync();
-  // Bucket members side by side (every key is in registers by now).
+  // Bucket members side by side (every key is in registers by now); buckets that start at
+  // rank k or later hold no winner and are left out.
 #pragma unroll
   for (int i = 0; i < KPT; ++i) {
     const uint32_t e = rank + i * NT;
-    if (e < m) tmp[bk[bs[i] >> 16] + (bs[i] & 0xFFFFu)] = v[i];
+    if (e < m) {
+      const uint32_t s0 = bk[bs[i] >> 16];
+      if (s0 < k) tmp[s0 + (bs[i] & 0xFFFFu)] = v[i];
+    }
   }
   gs.sync();
 #pragma unroll
   for (int i = 0; i < KPT; ++i) {
     const uint32_t e = rank + i * NT;
+    bs[i] = 0xFFFFFFFFu;
     if (e < m) {
-      const uint32_t b = bs[i] >> 16;
+      const uint32_t b = bs_bucket[i];
       const uint32_t s0 = bk[b];
-      const uint32_t nb = (b == 0 ? m : bk[b - 1]) - s0;
-      uint32_t r = s0;
-      for (uint32_t j = 0; j < nb; ++j) r += tmp[s0 + j] > v[i] ? 1u : 0u;
-      bs[i] = r;
+      if (s0 < k) {
+        const uint32_t nb = (b == 0 ? m : bk[b - 1]) - s0;
+        uint32_t r = s0;
+        for (uint32_t j = 0; j < nb; ++j) r += tmp[s0 + j] > v[i] ? 1u : 0u;
+        bs[i] = r;
+      }
     }
   }
   gs.sync();

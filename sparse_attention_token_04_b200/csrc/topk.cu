@@ -19,14 +19,13 @@ namespace dsa {
 
 constexpr int kSortBuf = sort_buffer_len(DSA_MAX_TOPK);
 
-// Prefill finish. The keys at or above the row's threshold (normally k plus a few hundred) are
-// collected in shared memory and ranked by a bucket sort: 4096 buckets of equal width in score
-// value between the smallest and largest collected score (the rounded fp32 map is monotone, so
-// a larger key never lands in a lower bucket), a suffix scan for each bucket's first rank, and
-// inside a bucket a key's rank is found by comparing it with the bucket's other keys. Keys with rank
-// below k are the top-k in order. When a bucket holds more than kBucketMax keys (heavy ties,
-// scores bunched in a sliver of their span) the row falls back to an exact radix select and a
-// merge sort.
+// Prefill finish. Every key a row's candidate buffer holds is at or above the row's threshold
+// (the lean pass appends only such keys, the exact pass compacts to them), so the buffer is the
+// candidate set itself. Persistent CTAs walk rows r, r + G, ...; while one row is ranked, the
+// next row's buffer is copied into the other half of shared memory with cp.async. The ranking
+// is group_bucket_rank (4096 value-linear buckets); a row with heavy ties (a bucket over
+// kBucketMax keys) or more keys than a staging buffer holds falls back to an exact radix select
+// and a merge sort. The k largest keys are written in order, padded with -1 / -inf.
 constexpr int kFinishThreads = 512;
 constexpr uint32_t kFinishTmp = 4608;
 constexpr int kFinishKPT = kFinishTmp / kFinishThreads;  // keys ranked per thread
@@ -34,141 +33,152 @@ constexpr int kFinishBuckets = 4096;
 constexpr uint32_t kBucketMax = 256;
 
 struct FinishSmem {
-  uint64_t tmp[kFinishTmp];      // collected keys, then ranked keys; merge-sort buffers
-  uint32_t bk[kFinishBuckets];   // bucket counts, then first ranks; radix histogram, then winners
+  uint64_t buf[2][kFinishTmp];   // staged candidates of the current and the next row
+  uint32_t bk[kFinishBuckets];   // bucket counts / radix histogram, then (select path) winners
   GroupScratch<kFinishThreads> sc;
-  uint32_t n_tmp;
+  uint32_t n[2];                 // candidates of the row staged in each buffer
   uint32_t big;
   uint32_t omin, omax;           // order-preserving score bits of the smallest / largest key
 };
 static_assert(kFinishTmp % kFinishThreads == 0, "keys per thread");
-static_assert(kFinishTmp >= 2u * static_cast<uint32_t>(kSortBuf), "merge-sort buffers in tmp");
+static_assert(kFinishTmp >= 2u * static_cast<uint32_t>(kSortBuf), "merge-sort buffers in a staging buffer");
 static_assert(kFinishBuckets * sizeof(uint32_t) >= DSA_MAX_TOPK * sizeof(uint64_t), "winners in bk");
 static_assert(kFinishBuckets >= kHistBins, "radix histogram in bk");
 
-__global__ void __launch_bounds__(kFinishThreads)
-    prefill_finish_kernel(const uint64_t* __restrict__ cand, const uint32_t* __restrict__ counts,
-                          const uint64_t* __restrict__ thr_in, uint32_t pitch, int topk,
-                          int32_t* __restrict__ out_idx, float* __restrict__ out_score) {
-  extern __shared__ uint8_t smem_raw[];
-  FinishSmem& sm = *reinterpret_cast<FinishSmem*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 15) & ~static_cast<uintptr_t>(15));
-  const GroupSync<kFinishThreads> gs{0};
-  const uint32_t rank = threadIdx.x, lane = rank & 31u, lt = (1u << lane) - 1u;
-  const size_t row = blockIdx.x;
-  const uint32_t k = static_cast<uint32_t>(topk);
-  const uint32_t segcap = pitch / 4u;
-  const uint64_t* buf = cand + row * pitch;
+struct RowSegments {
+  const uint64_t* buf;
+  uint32_t o1, o2, o3, n, segcap;
+  __device__ __forceinline__ const uint64_t* at(uint32_t e) const {
+    const uint32_t w = (e >= o1 ? 1u : 0u) + (e >= o2 ? 1u : 0u) + (e >= o3 ? 1u : 0u);
+    const uint32_t start = e >= o3 ? o3 : (e >= o2 ? o2 : (e >= o1 ? o1 : 0u));
+    return buf + w * segcap + (e - start);
+  }
+};
+
+__device__ __forceinline__ RowSegments row_segments(const uint64_t* cand, const uint32_t* counts,
+                                                    uint32_t pitch, size_t row) {
+  RowSegments r;
+  r.segcap = pitch / 4u;
+  r.buf = cand + row * pitch;
   uint32_t c[4];
 #pragma unroll
   for (int w = 0; w < 4; ++w) {
     const uint32_t v = __ldcg(counts + row * 4 + w);
-    c[w] = v < segcap ? v : segcap;
+    c[w] = v < r.segcap ? v : r.segcap;
   }
-  const uint32_t o1 = c[0], o2 = o1 + c[1], o3 = o2 + c[2], n = o3 + c[3];
-  const uint64_t thr = __ldcg(thr_in + row);
-  auto src_of = [&](uint32_t e) -> const uint64_t* {
-    const uint32_t w = (e >= o1 ? 1u : 0u) + (e >= o2 ? 1u : 0u) + (e >= o3 ? 1u : 0u);
-    const uint32_t start = e >= o3 ? o3 : (e >= o2 ? o2 : (e >= o1 ? o1 : 0u));
-    return buf + w * segcap + (e - start);
+  r.o1 = c[0];
+  r.o2 = r.o1 + c[1];
+  r.o3 = r.o2 + c[2];
+  r.n = r.o3 + c[3];
+  return r;
+}
+
+__global__ void __launch_bounds__(kFinishThreads, 2)
+    prefill_finish_kernel(const uint64_t* __restrict__ cand, const uint32_t* __restrict__ counts,
+                          uint32_t pitch, int rows, int topk, int32_t* __restrict__ out_idx,
+                          float* __restrict__ out_score) {
+  extern __shared__ uint8_t smem_raw[];
+  FinishSmem& sm = *reinterpret_cast<FinishSmem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 15) & ~static_cast<uintptr_t>(15));
+  const GroupSync<kFinishThreads> gs{0};
+  const uint32_t rank = threadIdx.x, lane = rank & 31u;
+  const uint32_t k = static_cast<uint32_t>(topk);
+  const int G = gridDim.x;
+
+  // Copies a row's candidates into buf[b] (one cp.async group per thread, possibly empty).
+  auto stage = [&](int row, int b) {
+    const RowSegments seg = row_segments(cand, counts, pitch, static_cast<size_t>(row));
+    if (seg.n <= kFinishTmp)
+      for (uint32_t e = rank; e < seg.n; e += kFinishThreads) cp_async_8(&sm.buf[b][e], seg.at(e));
+    cp_async_commit();
+    if (rank == 0) sm.n[b] = seg.n;
   };
+
   for (uint32_t b = rank; b < kFinishBuckets; b += kFinishThreads) sm.bk[b] = 0u;
-  if (rank == 0) {
-    sm.n_tmp = 0u;
-    sm.big = 0u;
-    sm.omin = 0xFFFFFFFFu;
-    sm.omax = 0u;
-  }
-  gs.sync();
-  // Collect the keys at or above the threshold, sixteen independent loads in flight per thread
-  // (the whole buffer in one round for up to 8192 entries), with their score range.
-  uint32_t lmin = 0xFFFFFFFFu, lmax = 0u;
-  for (uint32_t e0 = 0; e0 < n; e0 += 16 * kFinishThreads) {
-    uint64_t v[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const uint32_t e = e0 + i * kFinishThreads + rank;
-      v[i] = e < n ? __ldcg(src_of(e)) : 0ull;
+  if (static_cast<int>(blockIdx.x) < rows) stage(blockIdx.x, 0);
+  int i = 0;
+  for (int row = blockIdx.x; row < rows; row += G, ++i) {
+    const int b = i & 1;
+    // Prefetch the next row into the other buffer (free since the previous row's last barrier).
+    if (row + G < rows) stage(row + G, b ^ 1);
+    else cp_async_commit();
+    if (rank == 0) {
+      sm.omin = 0xFFFFFFFFu;
+      sm.omax = 0u;
     }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const bool take = v[i] != 0ull && v[i] >= thr;
-      const uint32_t mm = __ballot_sync(0xFFFFFFFFu, take);
-      if (mm) {
-        uint32_t base = 0;
-        if (lane == 0) base = atomicAdd(&sm.n_tmp, static_cast<uint32_t>(__popc(mm)));
-        base = __shfl_sync(0xFFFFFFFFu, base, 0);
-        const uint32_t pos = base + __popc(mm & lt);
-        if (take && pos < kFinishTmp) sm.tmp[pos] = v[i];
-        if (take) {
-          const uint32_t o = static_cast<uint32_t>(v[i] >> 32);
-          lmin = o < lmin ? o : lmin;
-          lmax = o > lmax ? o : lmax;
-        }
+    cp_async_wait<1>();  // this thread's copies of the current row have landed
+    gs.sync();
+    const uint32_t n = sm.n[b];
+    uint64_t* keys = sm.buf[b];
+    const uint64_t* res = keys;
+    bool padded = false;
+    uint32_t n_res = 0;
+    bool need_select = n > kFinishTmp;
+    if (!need_select && n > 0) {
+      uint32_t lmin = 0xFFFFFFFFu, lmax = 0u;
+      for (uint32_t e = rank; e < n; e += kFinishThreads) {
+        const uint32_t o = static_cast<uint32_t>(keys[e] >> 32);
+        lmin = o < lmin ? o : lmin;
+        lmax = o > lmax ? o : lmax;
       }
+      lmin = __reduce_min_sync(0xFFFFFFFFu, lmin);
+      lmax = __reduce_max_sync(0xFFFFFFFFu, lmax);
+      if (lane == 0) {
+        atomicMin(&sm.omin, lmin);
+        atomicMax(&sm.omax, lmax);
+      }
+      gs.sync();
+      if (group_bucket_rank<kFinishThreads, kFinishKPT, kFinishBuckets>(
+              keys, n, k, sm.omin, sm.omax, kBucketMax, sm.bk, &sm.big, sm.sc, gs, rank))
+        n_res = n < k ? n : k;
+      else
+        need_select = true;  // bk is zero again
     }
-  }
-  lmin = __reduce_min_sync(0xFFFFFFFFu, lmin);
-  lmax = __reduce_max_sync(0xFFFFFFFFu, lmax);
-  if (lane == 0 && lmax != 0u) {
-    atomicMin(&sm.omin, lmin);
-    atomicMax(&sm.omax, lmax);
-  }
-  gs.sync();
-  const uint32_t m = sm.n_tmp;
-  const uint64_t* res = sm.tmp;
-  bool padded = false;
-  uint32_t n_res = 0;
-  bool need_select = m > kFinishTmp;
-  auto tmp_at = [&](uint32_t i) { return sm.tmp[i]; };
-  if (!need_select && m > 0) {
-    if (group_bucket_rank<kFinishThreads, kFinishKPT, kFinishBuckets>(
-            sm.tmp, m, k, sm.omin, sm.omax, kBucketMax, sm.bk, &sm.big, sm.sc, gs, rank))
-      n_res = m < k ? m : k;
-    else
-      need_select = true;
-  }
-  if (need_select) {
-    // Exact radix select of the k-th key and a merge sort of the winners. bk is zero here.
-    uint64_t* win = reinterpret_cast<uint64_t*>(sm.bk);
-    uint32_t nw;
-    if (m <= kFinishTmp) {
-      const uint64_t T = m > k ? group_kth_threshold<kFinishThreads>(tmp_at, m, k, rank, sm.bk, sm.sc, gs) : 0ull;
-      nw = group_compact_ge<kFinishThreads>(
-          tmp_at, m, T, [&](uint32_t pos, uint64_t key) { if (pos < k) win[pos] = key; }, rank, sm.sc, gs);
-    } else {
-      auto key_at = [&](uint32_t e) {
-        const uint64_t v = __ldcg(src_of(e));
-        return v >= thr ? v : 0ull;
-      };
-      const uint64_t T = group_kth_threshold<kFinishThreads>(key_at, n, k, rank, sm.bk, sm.sc, gs);
-      nw = group_compact_ge<kFinishThreads>(
-          key_at, n, T, [&](uint32_t pos, uint64_t key) { if (pos < k) win[pos] = key; }, rank, sm.sc, gs);
+    if (need_select) {
+      // Exact radix select of the k-th key and a merge sort of the winners (bk is zero here).
+      uint64_t* win = reinterpret_cast<uint64_t*>(sm.bk);
+      uint32_t nw;
+      if (n <= kFinishTmp) {
+        auto key_at = [keys](uint32_t e) { return keys[e]; };
+        const uint64_t T = n > k ? group_kth_threshold<kFinishThreads>(key_at, n, k, rank, sm.bk, sm.sc, gs) : 0ull;
+        nw = group_compact_ge<kFinishThreads>(
+            key_at, n, T, [&](uint32_t pos, uint64_t key) { if (pos < k) win[pos] = key; }, rank, sm.sc, gs);
+      } else {
+        const RowSegments seg = row_segments(cand, counts, pitch, static_cast<size_t>(row));
+        auto key_at = [&](uint32_t e) { return __ldcg(seg.at(e)); };
+        const uint64_t T = group_kth_threshold<kFinishThreads>(key_at, n, k, rank, sm.bk, sm.sc, gs);
+        nw = group_compact_ge<kFinishThreads>(
+            key_at, n, T, [&](uint32_t pos, uint64_t key) { if (pos < k) win[pos] = key; }, rank, sm.sc, gs);
+      }
+      nw = nw < k ? nw : k;
+      res = group_merge_sort_desc<kFinishThreads>(
+          [&](uint32_t e) { return e < nw ? win[e] : 0ull; }, keys, keys + kSortBuf, sort_size(k), rank, gs);
+      padded = true;
+      n_res = nw;
     }
-    nw = nw < k ? nw : k;
-    res = group_merge_sort_desc<kFinishThreads>(
-        [&](uint32_t i) { return i < nw ? win[i] : 0ull; }, sm.tmp, sm.tmp + kSortBuf, sort_size(k),
-        rank, gs);
-    padded = true;
-    n_res = nw;
+    int32_t* oi = out_idx + static_cast<size_t>(row) * k;
+    float* os = out_score ? out_score + static_cast<size_t>(row) * k : nullptr;
+    for (uint32_t e = rank; e < k; e += kFinishThreads) {
+      const uint64_t key = e < n_res ? res[padded ? spad(e) : e] : 0ull;
+      oi[e] = key_index(key);
+      if (os) os[e] = key_score(key);
+    }
+    gs.sync();  // the row's buffers are free
+    for (uint32_t bb = rank; bb < kFinishBuckets; bb += kFinishThreads) sm.bk[bb] = 0u;
   }
-  int32_t* oi = out_idx + row * k;
-  float* os = out_score ? out_score + row * k : nullptr;
-  for (uint32_t i = rank; i < k; i += kFinishThreads) {
-    const uint64_t key = i < n_res ? res[padded ? spad(i) : i] : 0ull;
-    oi[i] = key_index(key);
-    if (os) os[i] = key_score(key);
-  }
+  cp_async_wait<0>();
 }
 
 dsa_status launch_prefill_finish(const uint64_t* cand, const uint32_t* counts,
                                  const uint64_t* thr, uint32_t pitch, int rows, int topk,
-                                 int32_t* out_idx, float* out_score, cudaStream_t stream) {
+                                 int32_t* out_idx, float* out_score, int num_sms, cudaStream_t stream) {
+  (void)thr;  // every buffered key is at or above the row's threshold already
   const size_t smem = sizeof(FinishSmem) + 16;
   if (cudaFuncSetAttribute(prefill_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return DSA_ERR_CUDA;
-  prefill_finish_kernel<<<rows, kFinishThreads, smem, stream>>>(cand, counts, thr, pitch, topk,
+  const int grid = rows < 2 * num_sms ? rows : 2 * num_sms;
+  prefill_finish_kernel<<<grid, kFinishThreads, smem, stream>>>(cand, counts, pitch, rows, topk,
                                                                 out_idx, out_score);
   return cuda_status(cudaGetLastError());
 }
