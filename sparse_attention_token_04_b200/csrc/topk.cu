@@ -190,79 +190,117 @@ dsa_status launch_prefill_finish(const uint64_t* cand, const uint32_t* counts,
 // the k-th largest key is a 6.5-sigma event, and otherwise at least k keys of the row are >= T.
 // A row with r >= n_s (short rows, n <= k) gets T = 0: every key is kept. (The lean pass checks
 // the count it actually appended and hands the rare failure to the exact pass.)
-constexpr int kSampleThreads = 256;
+// One warp per row: a radix select on the 64-bit keys with digits of up to 8 bits, starting at
+// the highest bit where the row's smallest and largest sampled key differ, with a warp-private
+// 256-bin histogram; no block-wide barrier.
+constexpr int kThrWarps = 8;
 
-__global__ void __launch_bounds__(kSampleThreads)
+__global__ void __launch_bounds__(32 * kThrWarps)
     prefill_sample_threshold_kernel(const uint64_t* __restrict__ cand, const uint32_t* __restrict__ counts,
-                                    uint64_t* __restrict__ thr, uint32_t seg_stride, int q_pos0, int Lk,
-                                    int topk, uint32_t stage_cap) {
-  extern __shared__ uint8_t smem_raw[];
-  uint64_t* stage = reinterpret_cast<uint64_t*>(smem_raw);  // stage_cap keys
-  __shared__ uint32_t hist[kHistBins];
-  __shared__ GroupScratch<kSampleThreads> sc;
-  const GroupSync<kSampleThreads> gs{0};
-  const uint32_t rank = threadIdx.x;
-  const size_t row = blockIdx.x;
-  const uint64_t* buf = cand + row * 4u * seg_stride;
+                                    uint64_t* __restrict__ thr, uint32_t seg_stride, int rows, int q_pos0,
+                                    int Lk, int topk) {
+  __shared__ uint32_t hist_all[kThrWarps][256];
+  const uint32_t lane = threadIdx.x & 31u, wi = threadIdx.x >> 5;
+  const int row = blockIdx.x * kThrWarps + static_cast<int>(wi);
+  if (row >= rows) return;  // warp-uniform; the block has no barrier
+  uint32_t* hist = hist_all[wi];
+  const uint64_t* buf = cand + static_cast<size_t>(row) * 4u * seg_stride;
   uint32_t c[4];
 #pragma unroll
   for (int w = 0; w < 4; ++w) {
-    const uint32_t v = __ldcg(counts + row * 4 + w);
+    const uint32_t v = __ldcg(counts + static_cast<size_t>(row) * 4 + w);
     c[w] = v < seg_stride ? v : seg_stride;
   }
   const uint32_t o1 = c[0], o2 = o1 + c[1], o3 = o2 + c[2], ns = o3 + c[3];
-  const int keys = min(q_pos0 + static_cast<int>(row) + 1, Lk);
+  const int keys = min(q_pos0 + row + 1, Lk);
   const double rho = static_cast<double>(topk) * ns / keys;
   const double rr = rho + 6.5 * sqrt(rho) + 1.0;
   if (rr >= static_cast<double>(ns)) {
-    if (rank == 0) thr[row] = 0ull;
+    if (lane == 0) thr[row] = 0ull;
     return;
   }
   const uint32_t r = static_cast<uint32_t>(ceil(rr));
-  auto src_at = [&](uint32_t e) {
+  auto key_at = [&](uint32_t e) {
     const uint32_t w = (e >= o1 ? 1u : 0u) + (e >= o2 ? 1u : 0u) + (e >= o3 ? 1u : 0u);
     const uint32_t start = e >= o3 ? o3 : (e >= o2 ? o2 : (e >= o1 ? o1 : 0u));
     return __ldcg(buf + w * seg_stride + (e - start));
   };
-  for (uint32_t b = rank; b < kHistBins; b += kSampleThreads) hist[b] = 0u;
-  uint64_t T;
-  if (ns <= stage_cap) {
-    // Stage the samples in shared memory (eight loads in flight per thread), select there.
-    for (uint32_t e0 = 0; e0 < ns; e0 += 8 * kSampleThreads) {
-      uint64_t v[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const uint32_t e = e0 + i * kSampleThreads + rank;
-        v[i] = e < ns ? src_at(e) : 0ull;
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const uint32_t e = e0 + i * kSampleThreads + rank;
-        if (e < ns) stage[e] = v[i];
-      }
-    }
-    gs.sync();
-    T = group_kth_threshold<kSampleThreads>([&](uint32_t e) { return stage[e]; }, ns, r, rank, hist, sc, gs);
-  } else {
-    gs.sync();
-    T = group_kth_threshold<kSampleThreads>(src_at, ns, r, rank, hist, sc, gs);
+  // Bits common to every sampled key are fixed from the start.
+  uint64_t mn = ~0ull, mx = 0ull;
+  for (uint32_t e = lane; e < ns; e += 32) {
+    const uint64_t v = key_at(e);
+    mn = v < mn ? v : mn;
+    mx = v > mx ? v : mx;
   }
-  if (rank == 0) thr[row] = T;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const uint64_t a = __shfl_xor_sync(0xFFFFFFFFu, mn, off), b = __shfl_xor_sync(0xFFFFFFFFu, mx, off);
+    mn = a < mn ? a : mn;
+    mx = b > mx ? b : mx;
+  }
+  int hb = 63 - __clzll(static_cast<long long>(mn ^ mx));
+  uint64_t mask = (hb >= 63) ? 0ull : ~((2ull << hb) - 1ull);
+  uint64_t prefix = mx & mask;
+  uint32_t need = r, taken = 0;
+  while (true) {
+    const int shift = hb >= 7 ? hb - 7 : 0;
+    const uint32_t dmask = (2u << (hb - shift)) - 1u;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) hist[lane * 8 + i] = 0u;
+    __syncwarp();
+    for (uint32_t e = lane; e < ns; e += 32) {
+      const uint64_t v = key_at(e);
+      if ((v & mask) == prefix) atomicAdd(&hist[static_cast<uint32_t>(v >> shift) & dmask], 1u);
+    }
+    __syncwarp();
+    // Bins 8*lane .. 8*lane+7; keys in higher bins come first.
+    uint32_t cb[8], local = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      cb[i] = hist[lane * 8 + i];
+      local += cb[i];
+    }
+    uint32_t suf = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t o = __shfl_down_sync(0xFFFFFFFFu, suf, off);
+      if (lane + off < 32) suf += o;
+    }
+    uint32_t acc = suf - local;
+    uint32_t hit = 0xFFFFFFFFu, hit_above = 0, hit_in = 0;
+#pragma unroll
+    for (int i = 7; i >= 0; --i) {
+      if (acc < need && acc + cb[i] >= need) {
+        hit = lane * 8 + i;
+        hit_above = acc;
+        hit_in = cb[i];
+      }
+      acc += cb[i];
+    }
+    const uint32_t bal = __ballot_sync(0xFFFFFFFFu, hit != 0xFFFFFFFFu);
+    const int src = __ffs(bal) - 1;  // exactly one lane holds the bin of the need-th key
+    const uint32_t bin = __shfl_sync(0xFFFFFFFFu, hit, src);
+    const uint32_t above = __shfl_sync(0xFFFFFFFFu, hit_above, src);
+    const uint32_t in_bin = __shfl_sync(0xFFFFFFFFu, hit_in, src);
+    need -= above;
+    taken += above;
+    prefix |= static_cast<uint64_t>(bin) << shift;
+    mask |= static_cast<uint64_t>(dmask) << shift;
+    __syncwarp();
+    if (taken + in_bin <= r || shift == 0) break;
+    hb = shift - 1;
+  }
+  if (lane == 0) thr[row] = prefix;
 }
 
 dsa_status launch_prefill_sample_threshold(const uint64_t* cand, const uint32_t* counts,
                                            uint64_t* thr, uint32_t seg_stride, int rows,
                                            int q_pos0, int Lk, int topk, uint32_t max_samples,
                                            cudaStream_t stream) {
-  // Shared staging for up to max_samples keys (at most 64 KB; longer samples select from global).
-  const uint32_t stage_cap = max_samples < 8192u ? max_samples : 8192u;
-  const size_t smem = static_cast<size_t>(stage_cap) * sizeof(uint64_t);
-  // The limit covers the dynamic part only; with the static histogram on top it can pass 48 KB.
-  if (cudaFuncSetAttribute(prefill_sample_threshold_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
-    return DSA_ERR_CUDA;
-  prefill_sample_threshold_kernel<<<rows, kSampleThreads, smem, stream>>>(cand, counts, thr, seg_stride,
-                                                                          q_pos0, Lk, topk, stage_cap);
+  (void)max_samples;
+  const int grid = (rows + kThrWarps - 1) / kThrWarps;
+  prefill_sample_threshold_kernel<<<grid, 32 * kThrWarps, 0, stream>>>(cand, counts, thr, seg_stride, rows,
+                                                                      q_pos0, Lk, topk);
   return cuda_status(cudaGetLastError());
 }
 
