@@ -226,11 +226,24 @@ __global__ void __launch_bounds__(32 * kThrWarps)
     return __ldcg(buf + w * seg_stride + (e - start));
   };
   // Bits common to every sampled key are fixed from the start.
+  // Eight independent loads in flight per lane in every pass over the samples.
+  constexpr int kBatch = 8;
   uint64_t mn = ~0ull, mx = 0ull;
-  for (uint32_t e = lane; e < ns; e += 32) {
-    const uint64_t v = key_at(e);
-    mn = v < mn ? v : mn;
-    mx = v > mx ? v : mx;
+  for (uint32_t e0 = 0; e0 < ns; e0 += 32 * kBatch) {
+    uint64_t v[kBatch];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const uint32_t e = e0 + i * 32 + lane;
+      v[i] = e < ns ? key_at(e) : 0ull;
+    }
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const uint32_t e = e0 + i * 32 + lane;
+      if (e < ns) {
+        mn = v[i] < mn ? v[i] : mn;
+        mx = v[i] > mx ? v[i] : mx;
+      }
+    }
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
@@ -248,9 +261,19 @@ __global__ void __launch_bounds__(32 * kThrWarps)
 #pragma unroll
     for (int i = 0; i < 8; ++i) hist[lane * 8 + i] = 0u;
     __syncwarp();
-    for (uint32_t e = lane; e < ns; e += 32) {
-      const uint64_t v = key_at(e);
-      if ((v & mask) == prefix) atomicAdd(&hist[static_cast<uint32_t>(v >> shift) & dmask], 1u);
+    for (uint32_t e0 = 0; e0 < ns; e0 += 32 * kBatch) {
+      uint64_t v[kBatch];
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        const uint32_t e = e0 + i * 32 + lane;
+        v[i] = e < ns ? key_at(e) : 0ull;
+      }
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        const uint32_t e = e0 + i * 32 + lane;
+        if (e < ns && (v[i] & mask) == prefix)
+          atomicAdd(&hist[static_cast<uint32_t>(v[i] >> shift) & dmask], 1u);
+      }
     }
     __syncwarp();
     // Bins 8*lane .. 8*lane+7; keys in higher bins come first.
