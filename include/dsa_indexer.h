@@ -136,8 +136,9 @@ DSA_API dsa_status dsa_indexer_decode(const uint8_t* q, const float* q_scale, co
  * not call cudaMalloc / cudaFree at step time (cudaFree synchronises the whole device). It
  * computes exactly what dsa_indexer_decode computes, with the same arguments except that,
  * instead of a workspace, its scratch is a fixed array inside the library:
- * DSA_WS_HEADER_BYTES + DSA_NOALLOC_MAX_SCORES * 4 + DSA_NOALLOC_MAX_REQUESTS * 8192 bytes
- * (18 MiB + 256 B), held on every GPU that loads the library until the process exits.
+ * DSA_WS_HEADER_BYTES + DSA_NOALLOC_MAX_SCORES * 4 + DSA_NOALLOC_MAX_REQUESTS * (8192 + 16 +
+ * 65536) bytes (34 MiB + 4352 B), held on every GPU that loads the library until the process
+ * exits.
  *   - B must not exceed DSA_NOALLOC_MAX_REQUESTS and B * max_blocks * block_size must not exceed
  *     DSA_NOALLOC_MAX_SCORES; a larger call returns DSA_ERR_UNSUPPORTED and enqueues nothing.
  *     Other errors are those of dsa_indexer_decode.

@@ -37,6 +37,7 @@ enum : uint32_t {
   DETAIL_WAIT_ACCEMPTY = 6,
   DETAIL_WAIT_DRAIN = 7,
   DETAIL_WAIT_SELFTEST = 8,
+  DETAIL_WAIT_SCORES = 9,
   DETAIL_BAD_BLOCK_TABLE = 16,
   DETAIL_BAD_SEQ_LEN = 17,
   DETAIL_BAD_INDEX = 18,
@@ -202,6 +203,16 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+// Plain bulk copy global -> shared (no tensor map): both addresses 16-byte aligned, bytes a
+// multiple of 16; completion is signalled on `bar` as transaction bytes.
+__device__ __forceinline__ void bulk_load_1d(void* smem_dst, const void* gsrc, uint32_t bytes,
+                                             uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {

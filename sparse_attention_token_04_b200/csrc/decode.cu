@@ -18,7 +18,7 @@
 
 namespace dsa {
 
-constexpr int kScoreBins = 2048;  // bins of the top 11 bits of an order-preserving fp32 key
+constexpr int kScoreBins = kDecodeScoreBins;  // bins of the top 11 bits of an order-preserving fp32 key
 
 template <int D>
 struct DCfg {
@@ -263,28 +263,26 @@ static dsa_status launch_decode_t(const DecodeLaunch& a) {
   p.n_blocks = a.n_blocks;
   p.max_len = max_len;
   uint8_t* base = static_cast<uint8_t*>(a.ws);
+  const DecodeLayout lay = decode_layout(a.B, static_cast<size_t>(a.B) * max_len);
   p.hdr = reinterpret_cast<WsHeader*>(base);
-  p.scores = reinterpret_cast<float*>(base + DSA_WS_HEADER_BYTES);
-  p.bins = reinterpret_cast<uint32_t*>(base + DSA_WS_HEADER_BYTES +
-                                       static_cast<size_t>(a.B) * max_len * sizeof(float));
+  p.scores = reinterpret_cast<float*>(base + lay.scores);
+  p.bins = reinterpret_cast<uint32_t*>(base + lay.bins);
   p.budget_ns = a.budget_ns;
-  if (cudaMemsetAsync(p.bins, 0, static_cast<size_t>(a.B) * kScoreBins * sizeof(uint32_t), a.stream) !=
-      cudaSuccess)
-    return DSA_ERR_CUDA;
+  // Histograms and collection state, cleared together.
+  if (cudaMemsetAsync(p.bins, 0, lay.cand - lay.bins, a.stream) != cudaSuccess) return DSA_ERR_CUDA;
   const int max_tiles = (max_len + C::BN - 1) / C::BN;
   dim3 grid((max_tiles + C::TPC - 1) / C::TPC, a.B);
   kern<<<grid, C::THREADS, smem, a.stream>>>(tq, tk, p);
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
-  return launch_decode_topk(p.scores, max_len, a.seq_lens, p.bins, a.B, a.topk, a.out_idx,
-                            a.out_score, a.ws, a.stream);
+  return launch_decode_topk(a.ws, lay, max_len, a.seq_lens, a.B, a.topk, a.out_idx, a.out_score,
+                            a.budget_ns, a.stream);
 }
 
 size_t decode_workspace_bytes(int B, int max_len, int H, int d, int topk) {
   (void)H;
   (void)d;
   (void)topk;
-  return DSA_WS_HEADER_BYTES + static_cast<size_t>(B) * max_len * sizeof(float) +
-         static_cast<size_t>(B) * kScoreBins * sizeof(uint32_t);
+  return decode_layout(B, static_cast<size_t>(B) * max_len).total;
 }
 
 dsa_status launch_decode(const DecodeLaunch& a) {

@@ -89,6 +89,28 @@ inline int prefill_queries_per_block(int H) { return 2 * (256 / H); }
 size_t prefill_workspace_bytes(int Lq, int H, int d, int topk, int num_sms);
 size_t decode_workspace_bytes(int B, int max_len, int H, int d, int topk);
 
+// Decode workspace after the header: the scores [B][max_len] fp32 the scoring kernel writes,
+// the per-request score histograms [B][kDecodeScoreBins] u32, the per-request collection state
+// [B][4] u32 (candidate count, largest ordered score, complement of the smallest, candidate
+// count the histogram predicts) and the per-request candidate keys [B][kDecodeCandCap] u64.
+// Histograms and state are adjacent so that one memset clears both.
+constexpr int kDecodeScoreBins = 2048;
+constexpr uint32_t kDecodeCandCap = 8192;
+struct DecodeLayout {
+  size_t scores, bins, state, cand, total;
+};
+constexpr size_t align_256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+// n_scores = B * max_len.
+constexpr DecodeLayout decode_layout(size_t B, size_t n_scores) {
+  DecodeLayout L{};
+  L.scores = DSA_WS_HEADER_BYTES;
+  L.bins = align_256(L.scores + n_scores * sizeof(float));
+  L.state = L.bins + B * kDecodeScoreBins * sizeof(uint32_t);
+  L.cand = align_256(L.state + B * 4 * sizeof(uint32_t));
+  L.total = L.cand + B * kDecodeCandCap * sizeof(uint64_t);
+  return L;
+}
+
 dsa_status launch_prefill(const PrefillLaunch& a);
 // Exact top-k of every row's candidate buffer, ordered and written to out_idx / out_score.
 dsa_status launch_prefill_finish(const uint64_t* cand, const uint32_t* counts,
@@ -101,9 +123,12 @@ dsa_status launch_prefill_sample_threshold(const uint64_t* cand, const uint32_t*
                                            int q_pos0, int Lk, int topk, uint32_t max_samples,
                                            cudaStream_t stream);
 dsa_status launch_decode(const DecodeLaunch& a);
-dsa_status launch_decode_topk(const float* scores, int max_len, const int32_t* seq_lens,
-                              const uint32_t* bins, int B, int topk, int32_t* out_idx,
-                              float* out_score, void* ws, cudaStream_t stream);
+// Exact top-k of every decode request's stored scores: a collection pass (several CTAs per
+// request) gathers the keys at or above the request's boundary histogram bin into its
+// candidate list, a rank pass (one CTA per request) orders them and writes the outputs.
+dsa_status launch_decode_topk(void* ws, const DecodeLayout& lay, int max_len,
+                              const int32_t* seq_lens, int B, int topk, int32_t* out_idx,
+                              float* out_score, uint64_t budget_ns, cudaStream_t stream);
 dsa_status launch_overlap(const int32_t* const* layer_idx, int32_t n_layers, int32_t rows,
                           int32_t topk, int32_t n_keys, uint64_t* out_counts, uint64_t* out_valid,
                           double* out_overlap, void* ws, cudaStream_t stream, int num_sms);

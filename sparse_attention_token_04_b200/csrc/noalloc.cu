@@ -4,8 +4,8 @@
 // application whose allocator owns all of the device memory, or a latency-critical decode loop
 // that must not call cudaMalloc / cudaFree at step time (cudaFree synchronises the whole
 // device). For them, dsa_indexer_decode_noalloc runs the same decode kernels with their scratch
-// (the status header and one fp32 score per cached key) placed in a fixed array that lives in
-// this file, instead of in a caller-provided workspace.
+// (the status header, one fp32 score per cached key and per-request selection state) placed
+// in a fixed array that lives in this file, instead of in a caller-provided workspace.
 //
 // The array is a file-scope __device__ variable, so every GPU that loads this library holds it
 // until the process exits. Its name is only a host-side stand-in for the device variable: host
@@ -20,10 +20,11 @@
 namespace dsa {
 namespace {
 
-// Status header, one fp32 score slot per cached key, and a 2048-bin score histogram per request.
-constexpr size_t kScratchBytes = DSA_WS_HEADER_BYTES +
-                                 static_cast<size_t>(DSA_NOALLOC_MAX_SCORES) * sizeof(float) +
-                                 static_cast<size_t>(DSA_NOALLOC_MAX_REQUESTS) * 2048 * sizeof(uint32_t);
+// The decode workspace of the largest call it takes: status header, one fp32 score slot per
+// cached key, and per request a 2048-bin score histogram, 16 bytes of collection state and
+// 8192 candidate keys.
+constexpr size_t kScratchBytes =
+    decode_layout(DSA_NOALLOC_MAX_REQUESTS, static_cast<size_t>(DSA_NOALLOC_MAX_SCORES)).total;
 
 // Zero at load time; the status header is cleared again at the end of every call, so each call
 // starts with a clean status (the decode launch itself clears the histograms it uses).

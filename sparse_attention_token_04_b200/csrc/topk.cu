@@ -5,12 +5,14 @@
 //                           fused scoring kernel left (four warp segments and a threshold),
 //                           ordered by (score descending, index ascending) and padded with
 //                           -1 / -inf.
-//   decode_topk_kernel    : per request, exact top-k of its n_b stored scores. The scoring
+//   decode_collect_kernel : per decode request, the candidates of its exact top-k. The scoring
 //                           kernel has already counted the request's scores in 2048 bins of
 //                           their order-preserving top 11 bits; the bin holding the k-th score
-//                           bounds the candidates, which one pass over the scores collects into
-//                           shared memory. The bucket ranking of the finish kernel orders them
-//                           (radix select + merge sort with heavy ties), same order and padding.
+//                           bounds the candidates, which several CTAs per request gather from
+//                           the stored scores into the request's candidate list.
+//   decode_rank_kernel    : per decode request, the candidates ordered by the bucket ranking of
+//                           the finish kernel (radix select + merge sort with heavy ties), same
+//                           order and padding.
 #include "common.cuh"
 #include "internal.h"
 #include "select.cuh"
@@ -327,8 +329,144 @@ dsa_status launch_prefill_sample_threshold(const uint64_t* cand, const uint32_t*
   return cuda_status(cudaGetLastError());
 }
 
+// Decode collection: CTA (c, b) takes scores [c * kCollectChunk, (c + 1) * kCollectChunk) of
+// request b. Four bulk copies bring its scores into shared memory while the CTA finds the
+// request's boundary bin from the histogram: the highest bin at or above which at least k
+// scores lie (bin 0 when the request has at most k keys: every key is a winner). The keys at or
+// above that bin are appended to the request's candidate list, one global atomic per CTA, and
+// the CTA's ordered score range is merged into the request's state.
+constexpr int kCollectThreads = 512;
+constexpr int kCollectParts = 4;
+constexpr int kCollectPart = 4096;  // scores per bulk copy
+constexpr int kCollectChunk = kCollectParts * kCollectPart;
+static_assert(kDecodeScoreBins == 4 * kCollectThreads, "four histogram bins per thread");
+static_assert(kCollectPart == 8 * kCollectThreads, "two float4 per thread per part");
+
+struct CollectSmem {
+  float4 v[kCollectChunk / 4];
+  uint64_t bar[kCollectParts];
+  GroupScratch<kCollectThreads> sc;
+  uint32_t bstar, n_cand, base, omin, omax;
+  int abort;
+};
+
+__global__ void __launch_bounds__(kCollectThreads)
+    decode_collect_kernel(const float* __restrict__ scores, int max_len,
+                          const int32_t* __restrict__ seq_lens, const uint32_t* __restrict__ bins,
+                          uint32_t* __restrict__ state, uint64_t* __restrict__ cand, int topk,
+                          WsHeader* hdr, uint64_t budget_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  CollectSmem& sm = *reinterpret_cast<CollectSmem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 15) & ~static_cast<uintptr_t>(15));
+  const GroupSync<kCollectThreads> gs{0};
+  const uint32_t rank = threadIdx.x, lane = rank & 31u;
+  const int req = blockIdx.y;
+  int n = seq_lens[req];  // a bad length is recorded by the rank pass
+  n = n < 1 ? 1 : (n > max_len ? max_len : n);
+  const uint32_t un = static_cast<uint32_t>(n), k = static_cast<uint32_t>(topk);
+  const uint32_t c0 = blockIdx.x * static_cast<uint32_t>(kCollectChunk);
+  if (c0 >= un) return;
+  const uint32_t len = min(un - c0, static_cast<uint32_t>(kCollectChunk));
+  const uint32_t parts = (len + kCollectPart - 1) / kCollectPart;
+  const float* src = scores + static_cast<size_t>(req) * max_len + c0;
+  if (rank == 0) {
+    for (uint32_t q = 0; q < parts; ++q) mbar_init(&sm.bar[q], 1);
+    fence_mbar_init();
+    // Every copy starts 16-byte aligned (rows of a multiple of 64 scores); the last one is
+    // rounded up to whole float4, which stays inside the row.
+    for (uint32_t q = 0; q < parts; ++q) {
+      const uint32_t cnt = min(len - q * kCollectPart, static_cast<uint32_t>(kCollectPart));
+      const uint32_t bytes = ((cnt + 3u) & ~3u) * static_cast<uint32_t>(sizeof(float));
+      mbar_arrive_expect_tx(&sm.bar[q], bytes);
+      bulk_load_1d(&sm.v[q * (kCollectPart / 4)], src + q * kCollectPart, bytes, &sm.bar[q]);
+    }
+    sm.abort = 0;
+    sm.omin = 0xFFFFFFFFu;
+    sm.omax = 0u;
+    sm.bstar = 0u;
+    sm.n_cand = un;
+  }
+  // Boundary bin from the request's histogram (complete: the scoring kernel has finished).
+  if (un > k) {
+    const uint4 h = __ldcg(reinterpret_cast<const uint4*>(bins + static_cast<size_t>(req) * kDecodeScoreBins) + rank);
+    const uint32_t c[4] = {h.x, h.y, h.z, h.w};
+    uint32_t acc = group_suffix_exclusive<kCollectThreads>(c[0] + c[1] + c[2] + c[3], rank, sm.sc.w, gs, nullptr);
+#pragma unroll
+    for (int i = 3; i >= 0; --i) {
+      if (acc < k && acc + c[i] >= k) {
+        sm.bstar = rank * 4u + static_cast<uint32_t>(i);
+        sm.n_cand = acc + c[i];
+      }
+      acc += c[i];
+    }
+  }
+  gs.sync();
+  const uint32_t bstar = sm.bstar, n_cand = sm.n_cand;
+  if (blockIdx.x == 0 && rank == 0) state[req * 4 + 3] = n_cand;
+  const bool collect = n_cand <= kDecodeCandCap;  // else the rank pass selects from the scores
+  const WaitCtl ctl{hdr, &sm.abort, budget_ns};
+
+  // Pass 1: mark this thread's candidates (bit 8q + 4i + j: part q, float4 i, lane j).
+  uint32_t mask = 0u, lmin = 0xFFFFFFFFu, lmax = 0u;
+  bool ok = true;
+  for (uint32_t q = 0; q < parts && collect; ++q) {
+    ok = mbar_wait(&sm.bar[q], 0, ctl, DETAIL_WAIT_SCORES);
+    if (!ok) break;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const uint32_t f4 = q * (kCollectPart / 4) + static_cast<uint32_t>(i) * kCollectThreads + rank;
+      const float4 v = sm.v[f4];
+      const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t o = float_to_ordered(vv[j] + 0.0f);
+        if (4u * f4 + j < len && (o >> 21) >= bstar) {
+          mask |= 1u << (8u * q + 4u * i + j);
+          lmin = min(lmin, o);
+          lmax = max(lmax, o);
+        }
+      }
+    }
+  }
+  ok = named_bar_and(0, kCollectThreads, ok);
+  if (collect && ok) {
+    // Pass 2: reserve this CTA's slice of the candidate list, then write the keys.
+    uint32_t total = 0;
+    const uint32_t off = group_prefix_exclusive<kCollectThreads>(__popc(mask), rank, sm.sc.w, gs, &total);
+    lmin = __reduce_min_sync(0xFFFFFFFFu, lmin);
+    lmax = __reduce_max_sync(0xFFFFFFFFu, lmax);
+    if (lane == 0 && lmax != 0u) {
+      atomicMin(&sm.omin, lmin);
+      atomicMax(&sm.omax, lmax);
+    }
+    gs.sync();
+    if (rank == 0 && total > 0) {
+      sm.base = atomicAdd(&state[req * 4 + 0], total);
+      atomicMax(&state[req * 4 + 1], sm.omax);
+      atomicMax(&state[req * 4 + 2], ~sm.omin);
+    }
+    gs.sync();
+    uint64_t* dst = cand + static_cast<size_t>(req) * kDecodeCandCap;
+    uint32_t pos = sm.base + off;
+    while (mask) {
+      const uint32_t bit = __ffs(mask) - 1u;
+      mask &= mask - 1u;
+      const uint32_t f4 = (bit >> 3) * (kCollectPart / 4) + ((bit >> 2) & 1u) * kCollectThreads + rank;
+      const float v = reinterpret_cast<const float*>(sm.v)[4u * f4 + (bit & 3u)];
+      if (pos < kDecodeCandCap) dst[pos] = make_key(v, c0 + 4u * f4 + (bit & 3u));
+      ++pos;
+    }
+  } else if (rank == 0) {
+    // Let every copy this CTA issued land before it exits (bounded).
+    for (uint32_t q = 0; q < parts; ++q) mbar_wait_drain(&sm.bar[q], 0, budget_ns);
+  }
+}
+
+// Decode rank: one CTA per request orders the request's candidates (group_bucket_rank; heavy
+// ties fall back to a radix select and a merge sort) and writes the k best, padded with -1 / -inf.
+// A request whose boundary bin holds too many keys for the candidate list is selected from its
+// stored scores directly.
 constexpr int kDecodeTopkThreads = 1024;
-constexpr uint32_t kDecodeCandCap = 8192;
 constexpr int kDecodeBuckets = 4096;
 
 struct DecodeTopkSmem {
@@ -337,21 +475,21 @@ struct DecodeTopkSmem {
   uint64_t cand[kDecodeCandCap];    // candidates, ranked in place; or the second sort buffer
   uint32_t hist[kHistBins];
   GroupScratch<kDecodeTopkThreads> sc;
-  uint32_t n_cand, big, omin, omax;
+  uint32_t big;
 };
 static_assert(kDecodeCandCap >= static_cast<uint32_t>(kSortBuf), "second sort buffer");
 static_assert(sizeof(uint64_t) * kSortBuf >= sizeof(uint32_t) * kDecodeBuckets, "bucket counts in a");
 
 __global__ void __launch_bounds__(kDecodeTopkThreads)
-    decode_topk_kernel(const float* __restrict__ scores, int max_len,
-                       const int32_t* __restrict__ seq_lens, const uint32_t* __restrict__ bins,
-                       int topk, int32_t* __restrict__ out_idx, float* __restrict__ out_score,
-                       WsHeader* hdr) {
+    decode_rank_kernel(const float* __restrict__ scores, int max_len,
+                       const int32_t* __restrict__ seq_lens, const uint32_t* __restrict__ state,
+                       const uint64_t* __restrict__ cand_all, int topk,
+                       int32_t* __restrict__ out_idx, float* __restrict__ out_score, WsHeader* hdr) {
   extern __shared__ uint8_t smem_raw[];
   DecodeTopkSmem& sm = *reinterpret_cast<DecodeTopkSmem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 15) & ~static_cast<uintptr_t>(15));
   const GroupSync<kDecodeTopkThreads> gs{0};
-  const uint32_t rank = threadIdx.x, lane = rank & 31u;
+  const uint32_t rank = threadIdx.x;
   const int req = blockIdx.x;
   int n = seq_lens[req];
   if (n < 1 || n > max_len) {
@@ -361,90 +499,24 @@ __global__ void __launch_bounds__(kDecodeTopkThreads)
   const float* row = scores + static_cast<size_t>(req) * max_len;
   auto key_at = [&](uint32_t e) { return make_key(__ldcg(row + e), e); };
   const uint32_t un = static_cast<uint32_t>(n), k = static_cast<uint32_t>(topk);
+  const uint4 st = __ldcg(reinterpret_cast<const uint4*>(state) + req);
+  const uint32_t n_cand = st.w;
   uint32_t* bk = reinterpret_cast<uint32_t*>(sm.a);
   for (uint32_t b = rank; b < static_cast<uint32_t>(kDecodeBuckets); b += kDecodeTopkThreads) bk[b] = 0u;
-  if (rank == 0) {
-    sm.n_cand = 0u;
-    sm.omin = 0xFFFFFFFFu;
-    sm.omax = 0u;
-  }
-
-  // Boundary bin: the highest bin where the count of scores at or above it reaches k (bin 0
-  // when the request has at most k keys: every key is a winner).
-  uint32_t bstar = 0, n_cand = un;
-  if (un > k) {
-    for (uint32_t b = rank; b < kHistBins; b += kDecodeTopkThreads)
-      sm.hist[b] = bins[static_cast<size_t>(req) * kHistBins + b];
-    gs.sync();
-    constexpr int BPT = kHistBins / kDecodeTopkThreads;
-    uint32_t local = 0;
-#pragma unroll
-    for (int i = 0; i < BPT; ++i) local += sm.hist[rank * BPT + i];
-    uint32_t acc = group_suffix_exclusive<kDecodeTopkThreads>(local, rank, sm.sc.w, gs, nullptr);
-#pragma unroll
-    for (int i = BPT - 1; i >= 0; --i) {
-      const uint32_t c = sm.hist[rank * BPT + i];
-      if (acc < k && acc + c >= k) {
-        sm.sc.w[kDecodeTopkThreads / 32] = rank * BPT + i;
-        sm.sc.w[kDecodeTopkThreads / 32 + 1] = acc + c;
-      }
-      acc += c;
-    }
-    gs.sync();
-    bstar = sm.sc.w[kDecodeTopkThreads / 32];
-    n_cand = sm.sc.w[kDecodeTopkThreads / 32 + 1];
-    gs.sync();
-  }
-  for (uint32_t b = rank; b < kHistBins; b += kDecodeTopkThreads) sm.hist[b] = 0u;  // selects below need it zero
-  gs.sync();
+  for (uint32_t b = rank; b < kHistBins; b += kDecodeTopkThreads) sm.hist[b] = 0u;  // selects need it zero
 
   const uint64_t* res = sm.cand;
   bool padded = false;
   uint32_t n_res = 0;
   if (n_cand <= kDecodeCandCap) {
-    // One pass: keys whose bin is at or above the boundary bin, 32 score loads in flight per
-    // thread (a 200000-key request in seven rounds), with their score range.
-    constexpr int kInFlight = 32;
-    uint32_t lmin = 0xFFFFFFFFu, lmax = 0u;
-    for (uint32_t e0 = 0; e0 < un; e0 += kInFlight * kDecodeTopkThreads) {
-      float v[kInFlight];
-#pragma unroll
-      for (int i = 0; i < kInFlight; ++i) {
-        const uint32_t e = e0 + i * kDecodeTopkThreads + rank;
-        v[i] = e < un ? __ldcg(row + e) : 0.0f;
-      }
-#pragma unroll
-      for (int i = 0; i < kInFlight; ++i) {
-        const uint32_t e = e0 + i * kDecodeTopkThreads + rank;
-        const uint64_t key = make_key(v[i], e);
-        const bool take = e < un && static_cast<uint32_t>(key >> 53) >= bstar;
-        const uint32_t m = __ballot_sync(0xFFFFFFFFu, take);
-        if (m) {
-          uint32_t base = 0;
-          if (lane == 0) base = atomicAdd(&sm.n_cand, static_cast<uint32_t>(__popc(m)));
-          base = __shfl_sync(0xFFFFFFFFu, base, 0);
-          const uint32_t pos = base + __popc(m & ((1u << lane) - 1u));
-          if (take && pos < kDecodeCandCap) sm.cand[pos] = key;
-          if (take) {
-            const uint32_t o = static_cast<uint32_t>(key >> 32);
-            lmin = o < lmin ? o : lmin;
-            lmax = o > lmax ? o : lmax;
-          }
-        }
-      }
-    }
-    lmin = __reduce_min_sync(0xFFFFFFFFu, lmin);
-    lmax = __reduce_max_sync(0xFFFFFFFFu, lmax);
-    if (lane == 0 && lmax != 0u) {
-      atomicMin(&sm.omin, lmin);
-      atomicMax(&sm.omax, lmax);
-    }
+    const uint32_t got = st.x < kDecodeCandCap ? st.x : kDecodeCandCap;
+    const uint64_t* src = cand_all + static_cast<size_t>(req) * kDecodeCandCap;
+    for (uint32_t e = rank; e < got; e += kDecodeTopkThreads) sm.cand[e] = __ldcg(src + e);
     gs.sync();
-    const uint32_t got = sm.n_cand < kDecodeCandCap ? sm.n_cand : kDecodeCandCap;
     if (got != n_cand && rank == 0) record_error(hdr, DSA_ERR_DEVICE, DETAIL_HIST_MISMATCH);
     if (got > 0 &&
         group_bucket_rank<kDecodeTopkThreads, kDecodeCandCap / kDecodeTopkThreads, kDecodeBuckets>(
-            sm.cand, got, k, sm.omin, sm.omax, 256u, bk, &sm.big, sm.sc, gs, rank)) {
+            sm.cand, got, k, ~st.z, st.y, 256u, bk, &sm.big, sm.sc, gs, rank)) {
       n_res = got < k ? got : k;
     } else {
       // Heavy ties: exact radix select over the candidates, then a merge sort.
@@ -462,6 +534,7 @@ __global__ void __launch_bounds__(kDecodeTopkThreads)
     }
   } else {
     // Too many keys share the boundary bin (heavy ties): radix select over global memory.
+    gs.sync();
     const uint64_t T = group_kth_threshold<kDecodeTopkThreads>(key_at, un, k, rank, sm.hist, sm.sc, gs);
     uint32_t nw = group_compact_ge<kDecodeTopkThreads>(
         key_at, un, T, [&](uint32_t pos, uint64_t key) { if (pos < k) sm.win[pos] = key; }, rank,
@@ -479,15 +552,29 @@ __global__ void __launch_bounds__(kDecodeTopkThreads)
   }
 }
 
-dsa_status launch_decode_topk(const float* scores, int max_len, const int32_t* seq_lens,
-                              const uint32_t* bins, int B, int topk, int32_t* out_idx,
-                              float* out_score, void* ws, cudaStream_t stream) {
+dsa_status launch_decode_topk(void* ws, const DecodeLayout& lay, int max_len,
+                              const int32_t* seq_lens, int B, int topk, int32_t* out_idx,
+                              float* out_score, uint64_t budget_ns, cudaStream_t stream) {
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  const float* scores = reinterpret_cast<const float*>(base + lay.scores);
+  const uint32_t* bins = reinterpret_cast<const uint32_t*>(base + lay.bins);
+  uint32_t* state = reinterpret_cast<uint32_t*>(base + lay.state);
+  uint64_t* cand = reinterpret_cast<uint64_t*>(base + lay.cand);
+  WsHeader* hdr = static_cast<WsHeader*>(ws);
+  const size_t csmem = sizeof(CollectSmem) + 16;
+  if (cudaFuncSetAttribute(decode_collect_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(csmem)) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  const dim3 cgrid((max_len + kCollectChunk - 1) / kCollectChunk, B);
+  decode_collect_kernel<<<cgrid, kCollectThreads, csmem, stream>>>(scores, max_len, seq_lens, bins,
+                                                                   state, cand, topk, hdr, budget_ns);
+  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
   const size_t smem = sizeof(DecodeTopkSmem) + 16;
-  if (cudaFuncSetAttribute(decode_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(decode_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return DSA_ERR_CUDA;
-  decode_topk_kernel<<<B, kDecodeTopkThreads, smem, stream>>>(
-      scores, max_len, seq_lens, bins, topk, out_idx, out_score, static_cast<WsHeader*>(ws));
+  decode_rank_kernel<<<B, kDecodeTopkThreads, smem, stream>>>(scores, max_len, seq_lens, state, cand,
+                                                              topk, out_idx, out_score, hdr);
   return cuda_status(cudaGetLastError());
 }
 
