@@ -447,12 +447,12 @@ def run_decode(args, world, rank, device, peaks):
                         "searched 1/4 pattern (12 indexer layers)",
             "value": pairs / (ms / 1e3), "unit": UNIT, "ms_per_step": ms / args.decode_steps,
             "steps": args.decode_steps, "keys_per_layer": keys,
-            "roofline": {"kernel": "dsa_indexer_decode (decode_indexer_kernel + decode_topk_kernel)",
+            "roofline": {"kernel": "dsa_indexer_decode (decode_indexer_kernel + decode_collect_kernel + decode_rank_kernel)",
                          "bound": "hbm", "achieved": gbs, "peak": float(peaks["hbm_gbs"]),
                          "unit": "GB/s", "frac": gbs / float(peaks["hbm_gbs"]), "traffic": None,
                          "algorithmic_per_launch": f"{bytes_per_launch} B (d+4 per key + per-request q/w/scale/table/out)",
                          "launch_ms": launch_ms},
-            "gpu_launches": 2 * n_full * args.decode_steps}
+            "gpu_launches": 3 * n_full * args.decode_steps}
 
 
 def cpu_baseline_prefill(layers, f_bufs, seconds):

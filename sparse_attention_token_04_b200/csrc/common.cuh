@@ -140,6 +140,15 @@ __device__ __forceinline__ float key_score(uint64_t key) {
   return key ? ordered_to_float(static_cast<uint32_t>(key >> 32)) : -__int_as_float(0x7f800000);
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream serialisation may
+// start while the kernel before it on the stream is still running; grid_dependency_wait blocks
+// until that kernel has completed and its memory is visible (immediately, when launched without
+// the attribute). grid_launch_dependents lets the next such kernel start before this one ends.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------------------------------
 // mbarrier
 // ------------------------------------------------------------------------------------------

@@ -346,6 +346,7 @@ __global__ void __launch_bounds__(192)
     if (j > 0) flush_hist(b - 1);
   }
   __syncthreads();
+  grid_launch_dependents();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 128);

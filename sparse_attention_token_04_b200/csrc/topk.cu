@@ -369,6 +369,9 @@ __global__ void __launch_bounds__(kCollectThreads)
   const uint32_t len = min(un - c0, static_cast<uint32_t>(kCollectChunk));
   const uint32_t parts = (len + kCollectPart - 1) / kCollectPart;
   const float* src = scores + static_cast<size_t>(req) * max_len + c0;
+  // Everything above reads only what was complete before the scoring kernel started; the
+  // scores and the histogram below are that kernel's output.
+  grid_dependency_wait();
   if (rank == 0) {
     for (uint32_t q = 0; q < parts; ++q) mbar_init(&sm.bar[q], 1);
     fence_mbar_init();
@@ -460,6 +463,7 @@ __global__ void __launch_bounds__(kCollectThreads)
     // Let every copy this CTA issued land before it exits (bounded).
     for (uint32_t q = 0; q < parts; ++q) mbar_wait_drain(&sm.bar[q], 0, budget_ns);
   }
+  grid_launch_dependents();
 }
 
 // Decode rank: one CTA per request orders the request's candidates (group_bucket_rank; heavy
@@ -499,11 +503,13 @@ __global__ void __launch_bounds__(kDecodeTopkThreads)
   const float* row = scores + static_cast<size_t>(req) * max_len;
   auto key_at = [&](uint32_t e) { return make_key(__ldcg(row + e), e); };
   const uint32_t un = static_cast<uint32_t>(n), k = static_cast<uint32_t>(topk);
-  const uint4 st = __ldcg(reinterpret_cast<const uint4*>(state) + req);
-  const uint32_t n_cand = st.w;
   uint32_t* bk = reinterpret_cast<uint32_t*>(sm.a);
   for (uint32_t b = rank; b < static_cast<uint32_t>(kDecodeBuckets); b += kDecodeTopkThreads) bk[b] = 0u;
   for (uint32_t b = rank; b < kHistBins; b += kDecodeTopkThreads) sm.hist[b] = 0u;  // selects need it zero
+  // The collection pass (and, before it, the scoring kernel) has completed past this point.
+  grid_dependency_wait();
+  const uint4 st = __ldcg(reinterpret_cast<const uint4*>(state) + req);
+  const uint32_t n_cand = st.w;
 
   const uint64_t* res = sm.cand;
   bool padded = false;
@@ -565,16 +571,32 @@ dsa_status launch_decode_topk(void* ws, const DecodeLayout& lay, int max_len,
   if (cudaFuncSetAttribute(decode_collect_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(csmem)) != cudaSuccess)
     return DSA_ERR_CUDA;
-  const dim3 cgrid((max_len + kCollectChunk - 1) / kCollectChunk, B);
-  decode_collect_kernel<<<cgrid, kCollectThreads, csmem, stream>>>(scores, max_len, seq_lens, bins,
-                                                                   state, cand, topk, hdr, budget_ns);
-  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+  // Both passes are launched as programmatic dependents of the kernel before them, so their
+  // launch and prologue overlap its last CTAs; each waits for it before reading its output.
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((max_len + kCollectChunk - 1) / kCollectChunk, B);
+  cfg.blockDim = dim3(kCollectThreads);
+  cfg.dynamicSmemBytes = csmem;
+  cfg.stream = stream;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, decode_collect_kernel, scores, max_len, seq_lens, bins, state, cand, topk,
+                         hdr, budget_ns) != cudaSuccess)
+    return DSA_ERR_CUDA;
   const size_t smem = sizeof(DecodeTopkSmem) + 16;
   if (cudaFuncSetAttribute(decode_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return DSA_ERR_CUDA;
-  decode_rank_kernel<<<B, kDecodeTopkThreads, smem, stream>>>(scores, max_len, seq_lens, state, cand,
-                                                              topk, out_idx, out_score, hdr);
+  cfg.gridDim = dim3(B);
+  cfg.blockDim = dim3(kDecodeTopkThreads);
+  cfg.dynamicSmemBytes = smem;
+  if (cudaLaunchKernelEx(&cfg, decode_rank_kernel, scores, max_len, seq_lens,
+                         static_cast<const uint32_t*>(state), static_cast<const uint64_t*>(cand), topk,
+                         out_idx, out_score, hdr) != cudaSuccess)
+    return DSA_ERR_CUDA;
   return cuda_status(cudaGetLastError());
 }
 
