@@ -171,6 +171,9 @@ __global__ void __launch_bounds__(192)
     if (lane == 0) {
       prefetch_tmap(&tmap_q);
       prefetch_tmap(&tmap_k);
+      // The key pages are read once; evicting them first keeps the scores this kernel writes
+      // in L2 for the collection pass that reads them next.
+      const uint64_t stream_policy = l2_policy_evict_first();
       uint32_t kiss[C::STAGES], qiss[C::QBUF];
       for (int s = 0; s < C::STAGES; ++s) kiss[s] = 0;
       for (int s = 0; s < C::QBUF; ++s) qiss[s] = 0;
@@ -197,10 +200,11 @@ __global__ void __launch_bounds__(192)
           const int lb0 = 2 * tile, lb1 = 2 * tile + 1;
           const bool two = lb1 < nblk;
           mbar_arrive_expect_tx(&sm.kfull[st], two ? 2 * C::PAGE_BYTES : C::PAGE_BYTES);
-          tma_load_2d(sm.k[st], &tmap_k, 0, phys_block(table, lb0, true) * C::PAGE, &sm.kfull[st]);
+          tma_load_2d_hint(sm.k[st], &tmap_k, 0, phys_block(table, lb0, true) * C::PAGE, &sm.kfull[st],
+                           stream_policy);
           if (two)
-            tma_load_2d(sm.k[st] + C::PAGE_BYTES, &tmap_k, 0, phys_block(table, lb1, true) * C::PAGE,
-                        &sm.kfull[st]);
+            tma_load_2d_hint(sm.k[st] + C::PAGE_BYTES, &tmap_k, 0, phys_block(table, lb1, true) * C::PAGE,
+                             &sm.kfull[st], stream_policy);
           ++kiss[st];
         }
       }
@@ -292,9 +296,9 @@ __global__ void __launch_bounds__(192)
       const int32_t* table = p.block_table + static_cast<size_t>(b) * p.max_blocks;
       // This thread's key scale, loaded one tile ahead.
       auto scale_of = [&](int s) {
-        return s < n ? __ldg(&p.k_scale_cache[static_cast<size_t>(phys_block(table, s / C::PAGE, false)) *
-                                                  C::PAGE +
-                                              (s % C::PAGE)])
+        return s < n ? __ldcs(&p.k_scale_cache[static_cast<size_t>(phys_block(table, s / C::PAGE, false)) *
+                                                   C::PAGE +
+                                               (s % C::PAGE)])
                      : 0.0f;
       };
       float sk_next = scale_of(t * C::BN + static_cast<int>(wl * 32u + lane));
