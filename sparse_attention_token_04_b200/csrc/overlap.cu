@@ -2,8 +2,8 @@
 //
 // Integer work bound by reading the N index tensors (N * rows * topk * 4 bytes, each byte once).
 // A CTA walks rows. For a row it marks every layer's indices in per-layer shared-memory bitmaps
-// over the row's index range, counts each pair (i <= j) as the popcount of the AND of the two
-// bitmaps, and clears the bitmaps. When the N bitmaps over [0, n_keys) do not fit in shared
+// over the row's index range (all of a row's loads in flight before the first mark), counts
+// each pair (i <= j) as the popcount of the AND of the two bitmaps, and clears the bitmaps. When the N bitmaps over [0, n_keys) do not fit in shared
 // memory, one bitmap at a time is built and the other layers' entries are probed against it.
 // Counts accumulate in shared 64-bit counters per CTA and are added to the output once per CTA;
 // a finishing kernel mirrors the upper triangle and forms C / V.
@@ -27,12 +27,24 @@ __device__ __forceinline__ unsigned long long* overlap_acc(uint8_t* smem) {
   return reinterpret_cast<unsigned long long*>(smem);
 }
 
-// All N bitmaps resident: bits[i][w], W words per layer.
+// All N bitmaps resident: bits[i][w], W words per layer. A row's indices are loaded for up to
+// kOvGroup layers at once (every load in flight before the first bitmap update), then marked.
+// With N <= kOvGroup (SMALL) each thread keeps its pair counts in registers across rows and
+// reduces them once at the end (and every kOvFlushRows rows, so a 32-bit count cannot wrap);
+// otherwise each row's pair counts are reduced per warp into the shared counters.
+constexpr int kOvGroup = 8;
+constexpr int kOvPerThread = DSA_MAX_TOPK / kOverlapThreads;  // indices per thread per layer
+constexpr int kOvPairs = kOvGroup * (kOvGroup + 1) / 2;
+constexpr int kOvFlushRows = 1 << 16;
+static_assert(DSA_MAX_TOPK % kOverlapThreads == 0, "indices per thread");
+
+template <bool SMALL>
 __global__ void __launch_bounds__(kOverlapThreads)
     overlap_bitmaps_kernel(const __grid_constant__ OverlapParams p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const int N = p.N;
-  const int npairs = N * (N + 1) / 2;
+  // Pair counters (SMALL: the kOvGroup x kOvGroup triangle, whatever N), then the valid count.
+  const int npairs = SMALL ? kOvPairs : N * (N + 1) / 2;
   unsigned long long* acc = overlap_acc(smem_raw);                        // [npairs + 1]
   int* row_max = reinterpret_cast<int*>(acc + npairs + 1);                 // [1] (+pad)
   uint32_t* bits = reinterpret_cast<uint32_t*>(row_max + 4);               // [N][W]
@@ -42,21 +54,49 @@ __global__ void __launch_bounds__(kOverlapThreads)
   if (threadIdx.x == 0) *row_max = -1;
   __syncthreads();
   const uint32_t lane = threadIdx.x & 31u;
+  uint32_t creg[kOvPairs];
+#pragma unroll
+  for (int q = 0; q < kOvPairs; ++q) creg[q] = 0u;
+  // Adds the register pair counts into the shared counters (all threads of the CTA).
+  auto flush_creg = [&]() {
+#pragma unroll
+    for (int q = 0; q < kOvPairs; ++q) {
+      uint32_t c = creg[q];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xFFFFFFFFu, c, o);
+      if (lane == 0 && c) atomicAdd(&acc[q], static_cast<unsigned long long>(c));
+      creg[q] = 0u;
+    }
+  };
+  int it = 0;
   for (int row = blockIdx.x; row < p.rows; row += gridDim.x) {
     const size_t off = static_cast<size_t>(row) * p.topk;
     int local_max = -1;
     uint32_t valid0 = 0;
-    for (int i = 0; i < N; ++i) {
-      const int32_t* Ti = p.layers[i] + off;
-      uint32_t* bi = bits + i * W;
-      for (int e = threadIdx.x; e < p.topk; e += kOverlapThreads) {
-        const int32_t v = __ldcs(&Ti[e]);
-        if (v >= 0 && v < p.n_keys) {
-          atomicOr(&bi[v >> 5], 1u << (v & 31));
-          local_max = v > local_max ? v : local_max;
-          if (i == 0) ++valid0;
-        } else if (v != -1) {
-          record_error(p.hdr, DSA_ERR_DEVICE, DETAIL_BAD_INDEX);
+    for (int i0 = 0; i0 < N; i0 += kOvGroup) {
+      int32_t v[kOvGroup][kOvPerThread];
+#pragma unroll
+      for (int ii = 0; ii < kOvGroup; ++ii) {
+        const int i = i0 + ii;
+#pragma unroll
+        for (int q = 0; q < kOvPerThread; ++q) {
+          const int e = static_cast<int>(threadIdx.x) + q * kOverlapThreads;
+          v[ii][q] = (i < N && e < p.topk) ? __ldcs(p.layers[i] + off + e) : -1;
+        }
+      }
+#pragma unroll
+      for (int ii = 0; ii < kOvGroup; ++ii) {
+        uint32_t* bi = bits + (i0 + ii) * W;
+#pragma unroll
+        for (int q = 0; q < kOvPerThread; ++q) {
+          const int32_t x = v[ii][q];
+          if (x >= 0 && x < p.n_keys) {
+            atomicOr(&bi[x >> 5], 1u << (x & 31));
+            local_max = x > local_max ? x : local_max;
+            if (i0 + ii == 0) ++valid0;
+          } else if (x != -1) {
+            record_error(p.hdr, DSA_ERR_DEVICE, DETAIL_BAD_INDEX);
+          }
         }
       }
     }
@@ -66,29 +106,62 @@ __global__ void __launch_bounds__(kOverlapThreads)
     if (lane == 0 && valid0) atomicAdd(&acc[npairs], static_cast<unsigned long long>(valid0));
     __syncthreads();
     const int wr = (*row_max >> 5) + 1;  // words that can hold a mark in this row
-    int pair = 0;
-    for (int i = 0; i < N; ++i) {
-      const uint32_t* bi = bits + i * W;
-      for (int j = i; j < N; ++j, ++pair) {
-        const uint32_t* bj = bits + j * W;
-        uint32_t c = 0;
-        for (int w = threadIdx.x; w < wr; w += kOverlapThreads) c += __popc(bi[w] & bj[w]);
+    if constexpr (SMALL) {
+      for (int w = threadIdx.x; w < wr; w += kOverlapThreads) {
+        uint32_t m[kOvGroup];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xFFFFFFFFu, c, o);
-        if (lane == 0 && c) atomicAdd(&acc[pair], static_cast<unsigned long long>(c));
+        for (int i = 0; i < kOvGroup; ++i) m[i] = i < N ? bits[i * W + w] : 0u;
+        int q = 0;
+#pragma unroll
+        for (int i = 0; i < kOvGroup; ++i)
+#pragma unroll
+          for (int j = i; j < kOvGroup; ++j, ++q) creg[q] += __popc(m[i] & m[j]);
+      }
+    } else {
+      int pair = 0;
+      for (int i = 0; i < N; ++i) {
+        const uint32_t* bi = bits + i * W;
+        for (int j = i; j < N; ++j, ++pair) {
+          const uint32_t* bj = bits + j * W;
+          uint32_t c = 0;
+          for (int w = threadIdx.x; w < wr; w += kOverlapThreads) c += __popc(bi[w] & bj[w]);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xFFFFFFFFu, c, o);
+          if (lane == 0 && c) atomicAdd(&acc[pair], static_cast<unsigned long long>(c));
+        }
       }
     }
     __syncthreads();
     for (int i = 0; i < N; ++i)
       for (int w = threadIdx.x; w < wr; w += kOverlapThreads) bits[i * W + w] = 0u;
     if (threadIdx.x == 0) *row_max = -1;
+    if constexpr (SMALL) {
+      if (++it == kOvFlushRows) {
+        flush_creg();
+        it = 0;
+      }
+    }
     __syncthreads();
   }
-  int pair = 0;
-  for (int i = 0; i < N; ++i)
-    for (int j = i; j < N; ++j, ++pair)
-      if (threadIdx.x == 0 && acc[pair]) atomicAdd(&p.counts[i * N + j], acc[pair]);
-  if (threadIdx.x == 0 && acc[npairs]) atomicAdd(p.valid, acc[npairs]);
+  if constexpr (SMALL) {
+    // Register pair q (i <= j over kOvGroup layers) is shared pair (i, j) over N layers.
+    flush_creg();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int q = 0;
+      for (int i = 0; i < kOvGroup; ++i)
+        for (int j = i; j < kOvGroup; ++j, ++q)
+          if (j < N && acc[q]) atomicAdd(&p.counts[i * N + j], acc[q]);
+      if (acc[npairs]) atomicAdd(p.valid, acc[npairs]);
+    }
+  } else {
+    __syncthreads();
+    int pair = 0;
+    for (int i = 0; i < N; ++i)
+      for (int j = i; j < N; ++j, ++pair)
+        if (threadIdx.x == 0 && acc[pair]) atomicAdd(&p.counts[i * N + j], acc[pair]);
+    if (threadIdx.x == 0 && acc[npairs]) atomicAdd(p.valid, acc[npairs]);
+  }
 }
 
 // One bitmap at a time (wide index ranges or many layers).
@@ -189,11 +262,14 @@ dsa_status launch_overlap(const int32_t* const* layer_idx, int32_t n_layers, int
   if (cudaMemsetAsync(out_valid, 0, sizeof(uint64_t), stream) != cudaSuccess) return DSA_ERR_CUDA;
   if (rows > 0) {
     const size_t words = static_cast<size_t>((n_keys + 31) / 32);
-    const size_t npairs = static_cast<size_t>(n_layers) * (n_layers + 1) / 2;
+    const size_t npairs = n_layers <= kOvGroup ? static_cast<size_t>(kOvPairs)
+                                               : static_cast<size_t>(n_layers) * (n_layers + 1) / 2;
     const size_t smem_all = (npairs + 1) * 8 + 16 + static_cast<size_t>(n_layers) * words * 4;
     dsa_status st;
-    if (smem_all <= kOverlapSmemBudget)
-      st = launch_overlap_kernel(overlap_bitmaps_kernel, p, smem_all, rows, stream, num_sms);
+    if (smem_all <= kOverlapSmemBudget && n_layers <= kOvGroup)
+      st = launch_overlap_kernel(overlap_bitmaps_kernel<true>, p, smem_all, rows, stream, num_sms);
+    else if (smem_all <= kOverlapSmemBudget)
+      st = launch_overlap_kernel(overlap_bitmaps_kernel<false>, p, smem_all, rows, stream, num_sms);
     else
       st = launch_overlap_kernel(overlap_probe_kernel, p, (nn + 1) * 8 + words * 4, rows, stream,
                                  num_sms);
