@@ -100,7 +100,8 @@ __global__ void __launch_bounds__(kOverlapThreads)
         }
       }
     }
-    if (local_max >= 0) atomicMax(row_max, local_max);
+    local_max = __reduce_max_sync(0xFFFFFFFFu, local_max);  // one shared atomic per warp
+    if (lane == 0 && local_max >= 0) atomicMax(row_max, local_max);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) valid0 += __shfl_xor_sync(0xFFFFFFFFu, valid0, o);
     if (lane == 0 && valid0) atomicAdd(&acc[npairs], static_cast<unsigned long long>(valid0));

@@ -102,7 +102,7 @@ def _random_rows(R, topk, n_keys, N, seed, base=None):
 
 
 @pytest.mark.parametrize("N,R,topk,n_keys", [(4, 300, 64, 300), (8, 100, 2048, 5000), (3, 1, 5, 5),
-                                                (12, 60, 256, 2000)])
+                                                (12, 60, 256, 2000), (5, 200, 130, 1000)])
 def test_overlap_counts_bit_exact(N, R, topk, n_keys):
     layers = _random_rows(R, topk, n_keys, N, seed=N * R)
     counts, valid, overlap = B.topk_overlap([torch.from_numpy(T).cuda() for T in layers], n_keys)
