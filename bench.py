@@ -449,10 +449,21 @@ def run_decode(args, world, rank, device, peaks):
             "steps": args.decode_steps, "keys_per_layer": keys,
             "roofline": {"kernel": "dsa_indexer_decode (decode_indexer_kernel + decode_collect_kernel + decode_rank_kernel)",
                          "bound": "hbm", "achieved": gbs, "peak": float(peaks["hbm_gbs"]),
-                         "unit": "GB/s", "frac": gbs / float(peaks["hbm_gbs"]), "traffic": None,
+                         "unit": "GB/s", "frac": gbs / float(peaks["hbm_gbs"]),
+                         "traffic": DECODE_SCORING_DRAM_BYTES_PER_KEY * keys,
+                         "traffic_source": "decode_indexer_kernel DRAM read+write per cached key from one ncu "
+                                           "capture of this workload (SpeedOfLight/MemoryWorkloadAnalysis "
+                                           "sections), times the keys of one launch",
                          "algorithmic_per_launch": f"{bytes_per_launch} B (d+4 per key + per-request q/w/scale/table/out)",
                          "launch_ms": launch_ms},
             "gpu_launches": 3 * n_full * args.decode_steps}
+
+
+# DRAM bytes (read + write) per cached key of decode_indexer_kernel, from one ncu capture of the
+# decode workload (32 requests, lengths U[10000, 200000]): 5.694 TB/s x 88.416 us = 5.034e8 B
+# over 3,737,801 keys (132 B of key and scale per key are algorithmic; the rest is the scores it
+# writes). Valid for the kernel as captured; a change to it makes this figure stale.
+DECODE_SCORING_DRAM_BYTES_PER_KEY = 5.034e8 / 3737801
 
 
 def cpu_baseline_prefill(layers, f_bufs, seconds):
