@@ -330,6 +330,7 @@ def dsa_selftest_wait_timeout(workspace: torch.Tensor, budget_ns: int, stream=No
 
 
 DSA_NOALLOC_MAX_SCORES = 4194304
+DSA_NOALLOC_MAX_REQUESTS = 256
 
 
 def dsa_indexer_decode_noalloc(q, q_scale, w, k_cache, k_scale_cache, block_table, seq_lens,

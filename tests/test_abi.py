@@ -76,3 +76,18 @@ def test_host_validation_without_gpu(lib):
     # unsupported head shape is reported before any launch
     st = lib.dsa_prefill_workspace_bytes(16, 32, 128, 8)
     assert st == 0
+
+
+def test_decode_workspace_size_matches_its_documented_layout(lib):
+    """Header + [B][max_len] fp32 scores + [B][2048] u32 histograms + [B] 16-byte collection
+    states + [B][8192] u64 candidate keys, sections 256-byte aligned; the no-alloc scratch is
+    that workspace for the largest call it takes (34 MiB + 4352 B, as the header states)."""
+    def align(x):
+        return (x + 255) // 256 * 256
+
+    for B, max_len in ((1, 64), (3, 640), (32, 200064), (256, 16384)):
+        want = align(binding.DSA_WS_HEADER_BYTES + B * max_len * 4) + B * 2048 * 4
+        want = align(want + B * 16) + B * 8192 * 8
+        assert binding.dsa_decode_workspace_bytes(B, max_len, 64, 128, 2048) == want, (B, max_len)
+    n_req, n_scores = binding.DSA_NOALLOC_MAX_REQUESTS, binding.DSA_NOALLOC_MAX_SCORES
+    assert binding.dsa_decode_workspace_bytes(n_req, n_scores // n_req, 64, 128, 2048) == 34 * 2**20 + 4352

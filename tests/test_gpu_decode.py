@@ -21,7 +21,13 @@ def run_decode(table, lens, layer, topk):
 
 
 @pytest.mark.parametrize("lens,topk", [([1, 63, 64, 65, 200, 3000, 2048, 2049], 2048),
-                                       ([5000, 777, 130], 100), ([12000, 9000], 2048)])
+                                       ([5000, 777, 130], 100), ([12000, 9000], 2048),
+                                       # more tiles than resident scoring CTAs: ranges that
+                                       # cross requests, and requests over one 16384-score
+                                       # collection slice
+                                       (decode_lengths(48, 1000, 24000, seed=11), 2048),
+                                       # many short requests: several request switches per CTA
+                                       (decode_lengths(200, 100, 2000, seed=12), 64)])
 def test_decode_vs_oracle(lens, topk):
     table, seq, layers = paged_decode_layers(lens, 64, 128, 1, seed=sum(lens))
     layer = next(layers)
