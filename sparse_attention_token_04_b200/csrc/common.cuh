@@ -204,7 +204,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
 }
 
 // ------------------------------------------------------------------------------------------
-// TMA (no multicast anywhere in this library)
+// TMA (every load fills only the issuing CTA's own shared memory)
 // ------------------------------------------------------------------------------------------
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int32_t x,
                                             int32_t y, uint64_t* bar) {
