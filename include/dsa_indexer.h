@@ -113,10 +113,13 @@ DSA_API dsa_status dsa_indexer_prefill(const uint8_t* q, const float* q_scale, c
  *                                                 are not read)
  *   seq_lens      [B]                            i32, 1 <= seq_lens[b] <= max_blocks*block_size
  *   out_idx       [B][topk] i32 logical positions;  out_score [B][topk] f32 or NULL
- * block_size must be 64. A block-table entry outside [0, n_blocks) or a bad length is
+ * block_size must be 64 and B at most DSA_DECODE_MAX_REQUESTS (else DSA_ERR_UNSUPPORTED, nothing
+ * enqueued). A block-table entry outside [0, n_blocks) or a bad length is
  * recorded as DSA_ERR_DEVICE (the request's keys are then read from block 0 / clamped).
  * workspace: >= dsa_decode_workspace_bytes(B, max_blocks*block_size, H, d, topk) bytes.
  * -------------------------------------------------------------------------------------*/
+#define DSA_DECODE_MAX_REQUESTS 65535
+
 DSA_API size_t dsa_decode_workspace_bytes(int32_t B, int32_t max_len, int32_t H, int32_t d,
                                           int32_t topk);
 

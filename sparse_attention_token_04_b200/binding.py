@@ -329,6 +329,7 @@ def dsa_selftest_wait_timeout(workspace: torch.Tensor, budget_ns: int, stream=No
                                            _stream(stream)), "dsa_selftest_wait_timeout")
 
 
+DSA_DECODE_MAX_REQUESTS = 65535
 DSA_NOALLOC_MAX_SCORES = 4194304
 DSA_NOALLOC_MAX_REQUESTS = 256
 

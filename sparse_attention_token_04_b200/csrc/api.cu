@@ -55,6 +55,7 @@ dsa_status check_decode(const uint8_t* q, const float* q_scale, const float* w,
   if (static_cast<int64_t>(max_blocks) * block_size > INT32_MAX) return DSA_ERR_INVALID;
   if (!aligned(q, 16) || !aligned(k_cache, 16)) return DSA_ERR_INVALID;
   if (!(H == 64 && d == 128) || block_size != 64 || topk > DSA_MAX_TOPK) return DSA_ERR_UNSUPPORTED;
+  if (B > DSA_DECODE_MAX_REQUESTS) return DSA_ERR_UNSUPPORTED;  // one grid row per request
   return DSA_OK;
 }
 

@@ -70,6 +70,11 @@ def test_host_validation_without_gpu(lib):
         st = lib.indexcache_run(pat, n, ctypes.byref(shape), arr, fb, 1, out, binding.AFTER_LAYER_FN(),
                                 None, None, 0, None)
         assert st == binding.DSA_ERR_INVALID, pat
+    # decode: more requests than one launch takes, rejected before anything is enqueued
+    fake = ctypes.c_void_p(1 << 20)
+    st = lib.dsa_indexer_decode(fake, fake, fake, fake, fake, 1, 64, fake, 1, fake, 65536, 64, 128, 8,
+                                fake, nul, nul, 0, nul)
+    assert st == binding.DSA_ERR_UNSUPPORTED
     # overlap: too many layers / no pointers
     ptrs = (ctypes.c_void_p * 1)()
     assert lib.topk_overlap(ptrs, 65, 1, 1, 1, None, None, None, None, 0, None) == binding.DSA_ERR_INVALID
