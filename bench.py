@@ -4,19 +4,22 @@
     python -m torch.distributed.run --nnodes=1 --nproc-per-node N --master-addr 127.0.0.1 \
         --master-port P bench.py --gpus N ...
 
-One step = one pass of the whole hot path over one synthetic batch: the 8-layer IndexCache
-prefill stack (L = 16384 tokens, H = 64 heads, d = 128, top-k = 2048, pattern FSFSFSFS, layer
-inputs correlated with rho = 0.9), i.e. four fused prefill indexer launches with streaming
-top-k whose index buffers the four Shared layers alias, followed by the 8 x 8 top-k overlap
-of all eight layers. Inputs are generated on the device before timing; at N > 1 every rank
-runs its own independent stack (weak scaling, no collective on the data path).
+One step = one 200000-token prefill through a 47-layer model under the searched 1/4 IndexCache
+pattern (12 Full layers), with the indexer of every Full layer run on H = 64 heads, d = 128,
+top-k = 2048 over rho = 0.9 correlated FP8 E4M3 layers. The prefill is chunked by 8192 queries
+the way a model runs it: chunk c passes through all 47 layers (one indexcache_run call: the 12
+Full layers launch the fused indexer, the 35 Shared layers alias the last Full layer's index
+buffer) before chunk c + 1 starts. Inputs (all 47 layers, 81 GB) are generated on the device
+before timing and are far larger than L2. `value` counts the causal (query, key) pairs the
+Full layers score and top-k per second. The same step under the all-F, FFFS and FSSS patterns
+is timed once each (extra keys), as are the 8-layer 16384-token IndexCache stack with its 8 x 8
+top-k overlap and the 47-layer decode step of 32 requests (extra keys "stack_16k", "decode").
 
-The decode workload (32 requests, cache lengths uniform in [10000, 200000], 47 layers with
-the searched 1/4 pattern = 12 indexer layers, paged 64-token blocks) is timed in the same run
-and reported under "decode". The CPU baseline is the oracle on a bounded sample of rows.
+At N > 1 every rank runs its own independently seeded copy of the workload (weak scaling, no
+collective on the data path).
 
-`--impl reference` times the oracle (the only reference implementation there is) on the same
-workload, a bounded sample of rows per step, on the host cores.
+`--impl reference` times the oracle (the only reference implementation there is) on a bounded
+sample of query rows of the same workload, on the host cores.
 """
 
 from __future__ import annotations
@@ -40,10 +43,14 @@ if ROOT not in sys.path:
 METRIC = "indexer q·k pairs scored+top-k'd/s (prefill, decode); % of FP8 / HBM roofline"
 UNIT = "pairs/s"
 
-PREFILL = dict(L=16384, H=64, d=128, topk=2048, n_layers=8, pattern="FSFSFSFS", seed=2)
+LONG = dict(L=200000, H=64, d=128, topk=2048, n_layers=47, chunk=8192, seed=5)
+STACK = dict(L=16384, H=64, d=128, topk=2048, n_layers=8, pattern="FSFSFSFS", seed=2)
 DECODE = dict(B=32, lo=10000, hi=200000, H=64, d=128, topk=2048, n_layers=47, seed=4)
 
 FP8_PER_BF16 = 2.0  # nominal dense FP8 / BF16 tensor throughput ratio on B200
+# Kernel launches of one dsa_indexer_prefill call with top-k 2048: sample pass, per-row sample
+# threshold, lean pass, exact pass (exits at once when the lean pass marked no block), finish.
+PREFILL_LAUNCHES_PER_CALL = 5
 
 
 # ------------------------------------------------------------------------------------------
@@ -176,223 +183,259 @@ def numpy_threads() -> int:
         return 1
 
 
-# ------------------------------------------------------------------------------------------
-# workloads
-# ------------------------------------------------------------------------------------------
-
-def make_prefill_stack(device, seed):
-    from synth import correlated_layers
-    cfg = PREFILL
-    layers = []
-    for l, lay in enumerate(correlated_layers(cfg["L"], cfg["H"], cfg["d"], cfg["n_layers"], seed,
-                                              device=device)):
-        layers.append(lay if cfg["pattern"][l] == "F" else None)
-    return layers
 
 
-def make_decode_stack(device, seed):
-    from synth import SEARCHED_QUARTER_PATTERN, decode_lengths, paged_decode_layers
-    cfg = DECODE
-    lens = decode_lengths(cfg["B"], cfg["lo"], cfg["hi"], seed)
-    table, seq, gen = paged_decode_layers(lens, cfg["H"], cfg["d"], cfg["n_layers"], seed, device=device)
-    layers = []
-    for l, lay in enumerate(gen):
-        layers.append(lay if SEARCHED_QUARTER_PATTERN[l] == "F" else None)
-    return lens, table, seq, layers
+def patterns_47():
+    from synth import SEARCHED_QUARTER_PATTERN
+    n = LONG["n_layers"]
+    return {"searched 1/4": SEARCHED_QUARTER_PATTERN, "all F": "F" * n,
+            "FFFS": ("FFFS" * 12)[:n], "FSSS": ("FSSS" * 12)[:n]}
 
 
-def prefill_dicts(layers):
-    return [None if l is None else {"q": l.q, "q_scale": l.q_scale, "w": l.w, "k": l.k,
-                                    "k_scale": l.k_scale} for l in layers]
-
-
-def decode_dicts(layers):
-    return [None if l is None else {"q": l.q, "q_scale": l.q_scale, "w": l.w, "k_cache": l.k_cache,
-                                    "k_scale_cache": l.k_scale_cache} for l in layers]
+def peak_tflops(peaks, sustained: bool) -> float:
+    key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
+    return FP8_PER_BF16 * float(peaks[key])
 
 
 # ------------------------------------------------------------------------------------------
-# our implementation
+# the 200000-token, 47-layer prefill (headline)
 # ------------------------------------------------------------------------------------------
 
-def run_ours(args, world, rank, local):
+class LongPrefill:
+    """Device-resident inputs of all 47 layers and the chunk-major IndexCache step."""
+
+    def __init__(self, device, seed):
+        from synth import correlated_layers
+        c = LONG
+        self.device = device
+        self.L, self.H, self.d, self.topk, self.chunk = c["L"], c["H"], c["d"], c["topk"], c["chunk"]
+        self.layers = list(correlated_layers(self.L, self.H, self.d, c["n_layers"], seed, device=device))
+        self.chunks = [(c0, min(self.L, c0 + self.chunk)) for c0 in range(0, self.L, self.chunk)]
+        # per chunk, every layer's views: queries of the chunk, keys before the chunk's end
+        self.views = [[{"q": l.q[c0:c1], "q_scale": l.q_scale[c0:c1], "w": l.w[c0:c1],
+                        "k": l.k[:c1], "k_scale": l.k_scale[:c1]} for l in self.layers]
+                      for c0, c1 in self.chunks]
+        from sparse_attention_token_04_b200 import binding as B
+        self.B = B
+        self.ws = torch.empty(B.dsa_prefill_workspace_bytes(self.chunk, self.H, self.d, self.topk),
+                              dtype=torch.uint8, device=device)
+        B.dsa_workspace_init(self.ws)
+        # the pages' single overwritten index cache: one chunk-sized buffer every F layer rewrites
+        self.out = torch.empty(self.chunk, self.topk, dtype=torch.int32, device=device)
+
+    def step(self, pattern, after_chunk_layer=None):
+        """One prefill of all chunks through all layers. after_chunk_layer(ci, l) is called after
+        layer l of chunk ci has been enqueued (host side), before the next layer can overwrite."""
+        for ci, (c0, c1) in enumerate(self.chunks):
+            views = [v if pattern[l] == "F" else None for l, v in enumerate(self.views[ci])]
+            cb = None
+            if after_chunk_layer is not None:
+                cb = (lambda ci_: (lambda l, p: after_chunk_layer(ci_, l)))(ci)
+            self.B.indexcache_run(pattern, views, self.topk, f_bufs=[self.out[: c1 - c0]],
+                                  q_pos0=c0, workspace=self.ws, after_layer=cb)
+
+    def pairs(self, pattern):
+        return pattern.count("F") * causal_pairs(self.L)
+
+    def calls(self, pattern):
+        return pattern.count("F") * len(self.chunks)
+
+
+def timed(stream, fn, n):
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def run_long(args, world, rank, device, peaks, peak_kind):
+    from synth import SEARCHED_QUARTER_PATTERN
+    stream = torch.cuda.current_stream()
+    lp = LongPrefill(device, rank_seed(LONG["seed"], rank))
+    pattern = SEARCHED_QUARTER_PATTERN
+    for _ in range(args.warmup):
+        lp.step(pattern)
+    torch.cuda.synchronize()
+    status = lp.B.dsa_read_device_status(lp.ws)
+    if status != (0, 0):
+        raise RuntimeError(f"device status after warm-up: {status}")
+
+    with ClockSampler(device.index) as clocks:
+        barrier(world, device)
+        torch.cuda.synchronize()
+        ms_total = timed(stream, lambda: lp.step(pattern), args.steps)
+        barrier(world, device)
+    clk = clocks.summary()
+    ms_max = max_over_ranks(ms_total, world, device)
+    ms_per_step = ms_max / args.steps
+    total_pairs = sum_over_ranks(lp.pairs(pattern) * args.steps, world, device)
+    value = total_pairs / (ms_max / 1e3)
+
+    # the same step under the other patterns, once each (S layers launch nothing)
+    pat = {}
+    for name, p in patterns_47().items():
+        ms = ms_per_step if p == pattern else timed(stream, lambda: lp.step(p), 1)
+        pat[name] = {"f_layers": p.count("F"), "ms": ms}
+    all_f = pat["all F"]["ms"]
+    for v in pat.values():
+        v["speedup_vs_all_f"] = all_f / v["ms"]
+
+    # per indexer layer: the 25 chunk calls of one F layer
+    n_full = pattern.count("F")
+    layer_ms = ms_per_step / n_full
+    flops_layer = 2.0 * lp.H * lp.d * causal_pairs(lp.L)
+    achieved = flops_layer / (layer_ms / 1e3) / 1e12
+    fp8_peak = peak_tflops(peaks, sustained=True)
+
+    e2e = run_long_e2e(args, world, lp, pattern, stream) if args.e2e_steps > 0 else None
+    return lp, {
+        "value": value, "ms_per_step": ms_per_step, "clocks": clk, "patterns": pat,
+        "gpu_launches": PREFILL_LAUNCHES_PER_CALL * lp.calls(pattern) * args.steps,
+        "roofline": {
+            "kernel": "dsa_indexer_prefill (sample, threshold, lean, exact-fallback and finish "
+                      "launches of the 25 chunk calls of one indexer layer, timed together)",
+            "bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
+            "frac": achieved / fp8_peak, "traffic": PREFILL_LEAN_TRAFFIC_PER_LAYER,
+            "peak_source": f"{peak_kind}: 2 x bf16_tflops_sustained (nominal FP8/BF16 ratio); the "
+                           "timed step runs for seconds",
+            "algorithmic_per_launch": f"2*H*d*L(L+1)/2 = {flops_layer:.4e} FLOP per indexer layer",
+            "launch_ms": layer_ms,
+            "traffic_source": PREFILL_LEAN_TRAFFIC_SOURCE},
+        "e2e": e2e,
+    }
+
+
+def run_long_e2e(args, world, lp, pattern, stream):
+    """The headline step end to end through the public API: every step copies the F layers'
+    inputs from pinned host memory to the device and every F layer's index rows back."""
+    f_layers = [l for l, c in enumerate(pattern) if c == "F"]
+    names = ("q", "q_scale", "w", "k", "k_scale")
+    host_in = {l: {n: getattr(lp.layers[l], n).cpu().pin_memory() for n in names} for l in f_layers}
+    host_out = {l: torch.empty(lp.L, lp.topk, dtype=torch.int32).pin_memory() for l in f_layers}
+    h2d = sum(t.numel() * t.element_size() for d in host_in.values() for t in d.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+
+    def after(ci, l):
+        if pattern[l] == "F":
+            c0, c1 = lp.chunks[ci]
+            host_out[l][c0:c1].copy_(lp.out[: c1 - c0], non_blocking=True)
+
+    def e2e_step():
+        for l in f_layers:
+            for n in names:
+                getattr(lp.layers[l], n).copy_(host_in[l][n], non_blocking=True)
+        lp.step(pattern, after_chunk_layer=after)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(world, lp.device)
+    ms = max_over_ranks(timed(stream, e2e_step, args.e2e_steps), world, lp.device)
+    pairs = sum_over_ranks(lp.pairs(pattern) * args.e2e_steps, world, lp.device)
+    del host_in, host_out
+    return {"value": pairs / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "steps": args.e2e_steps,
+            "ms_per_step": ms / args.e2e_steps}
+
+
+# DRAM bytes (read + write) per indexer layer of the 200000-token workload, scaled from one ncu
+# capture of the lean pass; None until a capture of the current kernel exists.
+PREFILL_LEAN_TRAFFIC_PER_LAYER = None
+PREFILL_LEAN_TRAFFIC_SOURCE = "not captured for the current kernel"
+
+
+# ------------------------------------------------------------------------------------------
+# the 8-layer 16384-token IndexCache stack with its top-k overlap (extra key)
+# ------------------------------------------------------------------------------------------
+
+def run_stack16k(args, world, rank, device, peaks, peak_kind):
     from sparse_attention_token_04_b200 import binding as B
-
-    device = torch.device("cuda", local)
-    torch.cuda.set_device(device)
-    init_dist(world, "nccl")
-    cfg = PREFILL
-    L, H, d, topk, pattern = cfg["L"], cfg["H"], cfg["d"], cfg["topk"], cfg["pattern"]
+    from synth import correlated_layers
+    c = STACK
+    L, H, d, topk, pattern = c["L"], c["H"], c["d"], c["topk"], c["pattern"]
     n_full = pattern.count("F")
     stream = torch.cuda.current_stream()
-
-    layers = make_prefill_stack(device, rank_seed(cfg["seed"], rank))
-    inputs = prefill_dicts(layers)
+    layers = [lay if pattern[l] == "F" else None for l, lay in
+              enumerate(correlated_layers(L, H, d, c["n_layers"], rank_seed(c["seed"], rank), device=device))]
+    inputs = [None if l is None else {"q": l.q, "q_scale": l.q_scale, "w": l.w, "k": l.k,
+                                      "k_scale": l.k_scale} for l in layers]
     f_bufs = [torch.empty(L, topk, dtype=torch.int32, device=device) for _ in range(n_full)]
-    shape_ws = B.dsa_prefill_workspace_bytes(L, H, d, topk)
-    ws = torch.empty(shape_ws, dtype=torch.uint8, device=device)
+    ws = torch.empty(B.dsa_prefill_workspace_bytes(L, H, d, topk), dtype=torch.uint8, device=device)
     B.dsa_workspace_init(ws)
-    ov_counts = torch.empty(cfg["n_layers"], cfg["n_layers"], dtype=torch.int64, device=device)
+    ov_counts = torch.empty(c["n_layers"], c["n_layers"], dtype=torch.int64, device=device)
     ov_valid = torch.empty(1, dtype=torch.int64, device=device)
-    ov = torch.empty(cfg["n_layers"], cfg["n_layers"], dtype=torch.float64, device=device)
+    ov = torch.empty(c["n_layers"], c["n_layers"], dtype=torch.float64, device=device)
     ov_ws = torch.zeros(256, dtype=torch.uint8, device=device)
-
-    layer_events = []
+    marks = []
 
     def on_layer(l, ptr):
-        if pattern[l] == "F" and layer_events is not None:
+        if pattern[l] == "F":
             ev = torch.cuda.Event(enable_timing=True)
             ev.record(stream)
-            layer_events[-1].append(ev)
+            marks[-1].append(ev)
 
     def step(record=False):
         if record:
-            ev0 = torch.cuda.Event(enable_timing=True)
-            ev0.record(stream)
-            layer_events.append([ev0])
+            ev = torch.cuda.Event(enable_timing=True)
+            ev.record(stream)
+            marks.append([ev])
         _, ptrs = B.indexcache_run(pattern, inputs, topk, f_bufs=f_bufs, workspace=ws,
                                    after_layer=on_layer if record else None)
-        if record:
-            evo = torch.cuda.Event(enable_timing=True)
-            evo.record(stream)
         B.topk_overlap_ptrs(ptrs, L, topk, L, ov_counts, ov_valid, ov, workspace=ov_ws)
         if record:
-            eve = torch.cuda.Event(enable_timing=True)
-            eve.record(stream)
-            layer_events[-1].extend([evo, eve])
+            ev = torch.cuda.Event(enable_timing=True)
+            ev.record(stream)
+            marks[-1].append(ev)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    status = B.dsa_read_device_status(ws)
-    if status != (0, 0):
-        raise RuntimeError(f"device status after warm-up: {status}")
+    if B.dsa_read_device_status(ws) != (0, 0):
+        raise RuntimeError("device status after the 16384-token stack warm-up")
+    barrier(world, device)
+    ms = max_over_ranks(timed(stream, lambda: step(True), args.stack_steps), world, device)
+    pf = [a.elapsed_time(b) for m in marks for a, b in zip(m[:n_full], m[1:n_full + 1])]
+    ovm = [m[-2].elapsed_time(m[-1]) for m in marks]
+    pf_ms, ov_ms = float(np.mean(pf)), float(np.mean(ovm))
+    flops = 2.0 * H * d * causal_pairs(L)
+    achieved = flops / (pf_ms / 1e3) / 1e12
+    peak = peak_tflops(peaks, sustained=False)
+    ov_bytes = c["n_layers"] * L * topk * 4
+    pairs = sum_over_ranks(n_full * causal_pairs(L) * args.stack_steps, world, device)
+    return {"workload": "IndexCache prefill stack: 8 layers, L=16384, H=64, d=128, k=2048, pattern "
+                        "FSFSFSFS (4 indexer layers), rho=0.9 correlated FP8 E4M3 layers, then the "
+                        "8x8 top-k overlap",
+            "value": pairs / (ms / 1e3), "unit": UNIT, "ms_per_step": ms / args.stack_steps,
+            "steps": args.stack_steps,
+            "prefill_call": {"launch_ms": pf_ms, "achieved_tflops": achieved, "peak_tflops": peak,
+                             "frac": achieved / peak,
+                             "peak_source": f"{peak_kind}: 2 x bf16_tflops (burst): a 2 ms call in a "
+                                            "short timed loop"},
+            "overlap_kernel": {"launch_ms": ov_ms, "bytes_per_launch": ov_bytes,
+                               "gbs": ov_bytes / (ov_ms / 1e3) / 1e9,
+                               "frac_hbm": ov_bytes / (ov_ms / 1e3) / 1e9 / float(peaks["hbm_gbs"])},
+            "gpu_launches": (PREFILL_LAUNCHES_PER_CALL * n_full + 2) * args.stack_steps}
 
-    pairs_per_step = n_full * causal_pairs(L)
-    # per prefill call: sample pass, sample threshold, lean pass, exact pass (exits at once when
-    # no block needs it), finish; then the two overlap kernels
-    launches_per_step = n_full * 5 + 2
-    with ClockSampler(local) as clocks:
-        barrier(world, device)
-        torch.cuda.synchronize()
-        t0 = torch.cuda.Event(enable_timing=True)
-        t1 = torch.cuda.Event(enable_timing=True)
-        t0.record(stream)
-        for _ in range(args.steps):
-            step(record=True)
-        t1.record(stream)
-        torch.cuda.synchronize()
-        barrier(world, device)
-    clk = clocks.summary()
-    ms_total = t0.elapsed_time(t1)
-    ms_max = max_over_ranks(ms_total, world, device)
-    ms_per_step = ms_max / args.steps
 
-    # per-launch times of the prefill indexer call and of the overlap
-    pf_ms, ov_ms = [], []
-    for evs in layer_events:
-        marks = evs[:-2]
-        for a, b in zip(marks[:-1], marks[1:]):
-            pf_ms.append(a.elapsed_time(b))
-        ov_ms.append(evs[-2].elapsed_time(evs[-1]))
-    pf_avg = float(np.mean(pf_ms))
-    ov_avg = float(np.mean(ov_ms))
-
-    total_pairs = sum_over_ranks(pairs_per_step * args.steps, world, device)
-    value = total_pairs / (ms_max / 1e3)
-
-    peaks, peak_kind = measured_peaks()
-    fp8_peak = FP8_PER_BF16 * float(peaks["bf16_tflops_sustained"])
-    flops_per_launch = 2.0 * H * d * causal_pairs(L)
-    achieved_tflops = flops_per_launch / (pf_avg / 1e3) / 1e12
-    ov_bytes = cfg["n_layers"] * L * topk * 4
-    ov_gbs = ov_bytes / (ov_avg / 1e3) / 1e9
-
-    # end to end through the public API with host buffers (pinned), copies timed
-    e2e = None
-    if args.e2e_steps > 0:
-        host_inputs = []
-        for lay in inputs:
-            host_inputs.append(None if lay is None else
-                               {k: v.cpu().pin_memory() for k, v in lay.items()})
-        host_out = [torch.empty(L, topk, dtype=torch.int32).pin_memory() for _ in range(n_full)]
-        host_ov = torch.empty(cfg["n_layers"], cfg["n_layers"], dtype=torch.float64).pin_memory()
-        h2d = sum(v.numel() * v.element_size() for lay in host_inputs if lay for v in lay.values())
-        d2h = sum(t.numel() * t.element_size() for t in host_out) + host_ov.numel() * 8
-
-        def e2e_step():
-            for lay, hl in zip(inputs, host_inputs):
-                if lay is not None:
-                    for k in lay:
-                        lay[k].copy_(hl[k], non_blocking=True)
-            _, ptrs = B.indexcache_run(pattern, inputs, topk, f_bufs=f_bufs, workspace=ws)
-            B.topk_overlap_ptrs(ptrs, L, topk, L, ov_counts, ov_valid, ov, workspace=ov_ws)
-            for hb, db in zip(host_out, f_bufs):
-                hb.copy_(db, non_blocking=True)
-            host_ov.copy_(ov, non_blocking=True)
-
-        e2e_step()
-        torch.cuda.synchronize()
-        barrier(world, device)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        barrier(world, device)
-        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
-        e2e_pairs = sum_over_ranks(pairs_per_step * args.e2e_steps, world, device)
-        e2e = {"value": e2e_pairs / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h), "steps": args.e2e_steps,
-               "ms_per_step": e2e_ms / args.e2e_steps}
-        del host_inputs, host_out
-
-    decode = run_decode(args, world, rank, device, peaks) if args.decode_steps > 0 else None
-
-    cpu = None
-    if rank == 0 and world == 1 and args.cpu_seconds > 0:
-        cpu = cpu_baseline_prefill(layers, f_bufs, args.cpu_seconds)
-
-    if rank == 0:
-        line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3", "data": "synthetic",
-            "config": {"workload": "IndexCache prefill stack: 8 layers, L=16384, H=64, d=128, "
-                                   "k=2048, pattern FSFSFSFS (4 indexer layers), rho=0.9 "
-                                   "correlated FP8 E4M3 layers, then the 8x8 top-k overlap",
-                       "L": L, "H": H, "d": d, "topk": topk, "n_layers": cfg["n_layers"],
-                       "pattern": pattern, "pairs_per_step_per_gpu": pairs_per_step,
-                       "l2": "inputs larger than L2 (4 x 134 MB of q read per step)",
-                       "parallelism": f"independent stack per GPU x{world}"},
-            "roofline": {"kernel": "dsa_indexer_prefill (sample, threshold, lean, exact-fallback and "
-                                   "finish launches, timed together)",
-                         "bound": "tensor", "achieved": achieved_tflops, "peak": fp8_peak,
-                         "unit": "TFLOP/s", "frac": achieved_tflops / fp8_peak, "traffic": None,
-                         "peak_source": f"{peak_kind}: 2 x bf16_tflops_sustained (nominal FP8/BF16 ratio)",
-                         "algorithmic_per_launch": f"2*H*d*L(L+1)/2 = {flops_per_launch:.4e} FLOP",
-                         "launch_ms": pf_avg},
-            "overlap_kernel": {"launch_ms": ov_avg, "bytes_per_launch": ov_bytes, "gbs": ov_gbs,
-                               "frac_hbm": ov_gbs / float(peaks["hbm_gbs"])},
-            "gpu_launches": launches_per_step * args.steps,
-            "clocks": clk,
-            "e2e": e2e,
-            "decode": decode,
-            "cpu_baseline": cpu,
-        }
-        print(json.dumps(line), flush=True)
-
+# ------------------------------------------------------------------------------------------
+# the 47-layer decode step (extra key)
+# ------------------------------------------------------------------------------------------
 
 def run_decode(args, world, rank, device, peaks):
     from sparse_attention_token_04_b200 import binding as B
-    from synth import SEARCHED_QUARTER_PATTERN
+    from synth import SEARCHED_QUARTER_PATTERN, decode_lengths, paged_decode_layers
 
     cfg = DECODE
-    lens, table, seq, layers = make_decode_stack(device, rank_seed(cfg["seed"], rank))
-    inputs = decode_dicts(layers)
+    seed = rank_seed(cfg["seed"], rank)
+    lens = decode_lengths(cfg["B"], cfg["lo"], cfg["hi"], seed)
+    table, seq, gen = paged_decode_layers(lens, cfg["H"], cfg["d"], cfg["n_layers"], seed, device=device)
     pattern = SEARCHED_QUARTER_PATTERN
+    layers = [lay if pattern[l] == "F" else None for l, lay in enumerate(gen)]
+    inputs = [None if l is None else {"q": l.q, "q_scale": l.q_scale, "w": l.w, "k_cache": l.k_cache,
+                                      "k_scale_cache": l.k_scale_cache} for l in layers]
     n_full = pattern.count("F")
     topk = cfg["topk"]
     f_bufs = [torch.empty(cfg["B"], topk, dtype=torch.int32, device=device) for _ in range(n_full)]
@@ -425,15 +468,7 @@ def run_decode(args, world, rank, device, peaks):
     if status != (0, 0):
         raise RuntimeError(f"decode device status after warm-up: {status}")
     barrier(world, device)
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(args.decode_steps):
-        step(record=True)
-    t1.record(stream)
-    torch.cuda.synchronize()
-    barrier(world, device)
-    ms = max_over_ranks(t0.elapsed_time(t1), world, device)
+    ms = max_over_ranks(timed(stream, lambda: step(True), args.decode_steps), world, device)
     keys = sum(lens)
     pairs = sum_over_ranks(keys * n_full * args.decode_steps, world, device)
     per = [a.elapsed_time(b) for evs in marks for a, b in zip(evs[:-1], evs[1:])]
@@ -447,50 +482,141 @@ def run_decode(args, world, rank, device, peaks):
                         "searched 1/4 pattern (12 indexer layers)",
             "value": pairs / (ms / 1e3), "unit": UNIT, "ms_per_step": ms / args.decode_steps,
             "steps": args.decode_steps, "keys_per_layer": keys,
-            "roofline": {"kernel": "dsa_indexer_decode (decode_indexer_kernel + decode_collect_kernel + decode_rank_kernel)",
+            "roofline": {"kernel": "dsa_indexer_decode (decode_indexer_kernel + decode_collect_kernel "
+                                   "+ decode_rank_kernel)",
                          "bound": "hbm", "achieved": gbs, "peak": float(peaks["hbm_gbs"]),
                          "unit": "GB/s", "frac": gbs / float(peaks["hbm_gbs"]),
-                         "traffic": DECODE_SCORING_DRAM_BYTES_PER_KEY * keys,
-                         "traffic_source": "decode_indexer_kernel DRAM read+write per cached key from one ncu "
-                                           "capture of this workload (SpeedOfLight/MemoryWorkloadAnalysis "
-                                           "sections), times the keys of one launch",
-                         "algorithmic_per_launch": f"{bytes_per_launch} B (d+4 per key + per-request q/w/scale/table/out)",
+                         "traffic": (None if DECODE_SCORING_DRAM_BYTES_PER_KEY is None
+                                     else DECODE_SCORING_DRAM_BYTES_PER_KEY * keys),
+                         "traffic_source": DECODE_TRAFFIC_SOURCE,
+                         "algorithmic_per_launch": f"{bytes_per_launch} B (d+4 per key + per-request "
+                                                   "q/w/scale/table/out)",
                          "launch_ms": launch_ms},
             "gpu_launches": 3 * n_full * args.decode_steps}
 
 
-# DRAM bytes (read + write) per cached key of decode_indexer_kernel, from one ncu capture of the
-# decode workload (32 requests, lengths U[10000, 200000]): 5.694 TB/s x 88.416 us = 5.034e8 B
-# over 3,737,801 keys (132 B of key and scale per key are algorithmic; the rest is the scores it
-# writes). Valid for the kernel as captured; a change to it makes this figure stale.
+# DRAM bytes (read + write) per cached key of decode_indexer_kernel from one ncu capture of this
+# workload, or None when the kernel changed after the capture.
 DECODE_SCORING_DRAM_BYTES_PER_KEY = 5.034e8 / 3737801
+DECODE_TRAFFIC_SOURCE = ("decode_indexer_kernel DRAM read+write per cached key from one ncu capture "
+                         "of this workload (SpeedOfLight/MemoryWorkloadAnalysis sections), times the "
+                         "keys of one launch")
 
 
-def cpu_baseline_prefill(layers, f_bufs, seconds):
-    """The oracle, as it stands, on sampled rows of the first F layer; checks those rows of
-    the GPU output on the way."""
-    import oracle.dsa_oracle as O
+# ------------------------------------------------------------------------------------------
+# CPU baseline: the oracle on sampled rows of the same workload
+# ------------------------------------------------------------------------------------------
+
+def cpu_baseline_long(lp, seconds):
+    """The C++ oracle, as it stands, on uniformly drawn query rows of the first indexer layer of
+    the headline workload: single-threaded (the plain oracle) for half the time, then the same
+    per-row function on nproc threads over rows. Every row it computes is also compared with
+    the GPU's row."""
+    import oracle.cpp_oracle as C
     sys.path.insert(0, os.path.join(ROOT, "tests"))
     from parity import check_row
+    from sparse_attention_token_04_b200 import binding as B
 
-    lay = layers[0].numpy()
-    L, topk = PREFILL["L"], PREFILL["topk"]
-    gpu = f_bufs[0].cpu().numpy()
+    lay = lp.layers[0]
+    k_h, ks_h = lay.k.cpu().numpy(), lay.k_scale.cpu().numpy()
     rng = np.random.default_rng(0)
-    pairs = 0
-    rows = 0
-    t0 = time.perf_counter()
-    while time.perf_counter() - t0 < seconds:
-        t = int(rng.integers(0, L))
-        r = O.prefill_rows(lay, topk, [t])[0]
-        check_row(gpu[t], None, r, topk)
-        pairs += t + 1
-        rows += 1
-    el = time.perf_counter() - t0
-    return {"value": pairs / el, "unit": UNIT, "cores": numpy_threads(), "kind": "oracle",
-            "sample": f"{rows} uniformly drawn query rows of indexer layer 0 of the same stack "
-                      f"({pairs} causal pairs, {el:.1f} s); GPU rows checked against it",
-            "host_nproc": os.cpu_count()}
+    rows = sorted({int(t) for t in rng.integers(0, lp.L, size=2048)})
+    gpu = {}
+    out = torch.empty(lp.chunk, lp.topk, dtype=torch.int32, device=lp.device)
+    for c0, c1 in lp.chunks:
+        want = [t for t in rows if c0 <= t < c1]
+        if not want:
+            continue
+        B.dsa_indexer_prefill(lay.q[c0:c1], lay.q_scale[c0:c1], lay.w[c0:c1], lay.k[:c1],
+                              lay.k_scale[:c1], lp.topk, q_pos0=c0, out_idx=out[: c1 - c0],
+                              want_score=False, workspace=lp.ws)
+        sel = out[torch.tensor([t - c0 for t in want], device=lp.device)].cpu().numpy()
+        for i, t in enumerate(want):
+            gpu[t] = sel[i]
+    order = [int(t) for t in rng.permutation(rows)]
+    pos_all = torch.tensor(order, device=lp.device)
+    q_h = lay.q[pos_all].cpu().numpy()
+    qs_h = lay.q_scale[pos_all].cpu().numpy()
+    w_h = lay.w[pos_all].cpu().numpy()
+    nproc = os.cpu_count() or 1
+
+    def run(first, count, threads):
+        sl = slice(first, first + count)
+        res = C.prefill_positions(q_h[sl], qs_h[sl], w_h[sl], k_h, ks_h, order[sl], lp.topk,
+                                  n_threads=threads)
+        for r in res:
+            check_row(gpu[r.t], None, r, lp.topk)
+        return sum(r.t + 1 for r in res)
+
+    nxt = 0
+    res = {}
+    for name, threads, batch in (("single", 1, 1), ("all", nproc, nproc)):
+        pairs = n = 0
+        t0 = time.perf_counter()
+        while nxt + batch <= len(order) and time.perf_counter() - t0 < seconds / 2:
+            pairs += run(nxt, batch, threads)
+            nxt += batch
+            n += batch
+        res[name] = (pairs, n, time.perf_counter() - t0)
+    p1, n1, e1 = res["single"]
+    pa, na, ea = res["all"]
+    return {"value": p1 / e1, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{n1} uniformly drawn query rows of indexer layer 0 of the 200000-token "
+                      f"workload ({p1} causal pairs, {e1:.1f} s) through the plain single-threaded "
+                      "C++ oracle; the GPU's rows checked against it",
+            "all_cores": {"value": pa / ea, "unit": UNIT, "cores": nproc,
+                          "sample": f"{na} more rows ({pa} pairs, {ea:.1f} s), the same per-row "
+                                    f"oracle on {nproc} threads over rows; checked the same way"},
+            "host_nproc": nproc}
+
+
+# ------------------------------------------------------------------------------------------
+# our implementation
+# ------------------------------------------------------------------------------------------
+
+def run_ours(args, world, rank, local):
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    init_dist(world, "nccl")
+    peaks, peak_kind = measured_peaks()
+
+    lp, long = run_long(args, world, rank, device, peaks, peak_kind)
+    cpu = None
+    if rank == 0 and world == 1 and args.cpu_seconds > 0:
+        cpu = cpu_baseline_long(lp, args.cpu_seconds)
+    del lp
+    torch.cuda.empty_cache()
+    stack = run_stack16k(args, world, rank, device, peaks, peak_kind) if args.stack_steps > 0 else None
+    decode = run_decode(args, world, rank, device, peaks) if args.decode_steps > 0 else None
+
+    if rank == 0:
+        c = LONG
+        line = {
+            "metric": METRIC, "value": long["value"], "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": long["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp8_e4m3", "data": "synthetic",
+            "config": {"workload": "200000-token prefill through 47 layers, searched 1/4 IndexCache "
+                                   "pattern (12 indexer layers), H=64, d=128, k=2048, rho=0.9 "
+                                   "correlated FP8 E4M3 layers, chunks of 8192 queries (chunk-major: "
+                                   "each chunk through all layers via one indexcache_run)",
+                       "L": c["L"], "H": c["H"], "d": c["d"], "topk": c["topk"],
+                       "n_layers": c["n_layers"], "chunk": c["chunk"],
+                       "pattern": patterns_47()["searched 1/4"],
+                       "pairs_per_step_per_gpu": 12 * causal_pairs(c["L"]),
+                       "l2": "inputs larger than L2 (12 x 1.64 GB of q read per step)",
+                       "parallelism": f"independent workload per GPU x{world}"},
+            "roofline": long["roofline"],
+            "patterns": long["patterns"],
+            "gpu_launches": long["gpu_launches"] + (stack["gpu_launches"] if stack else 0)
+            + (decode["gpu_launches"] if decode else 0),
+            "clocks": long["clocks"],
+            "e2e": long["e2e"],
+            "stack_16k": stack,
+            "decode": decode,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
 
 
 # ------------------------------------------------------------------------------------------
@@ -498,23 +624,30 @@ def cpu_baseline_prefill(layers, f_bufs, seconds):
 # ------------------------------------------------------------------------------------------
 
 def run_reference(args, world, rank):
+    """The C++ oracle on the host cores (nproc threads over rows), on uniformly drawn query
+    rows of the headline workload's shape: each step scores ref_rows rows at uniformly drawn
+    positions of a 200000-key layer. The oracle's cost per row depends only on its position."""
     if rank != 0:
         return
-    import oracle.dsa_oracle as O
-    from synth import correlated_layers
+    import oracle.cpp_oracle as C
+    from synth import gaussian_layer
 
-    cfg = PREFILL
-    L, H, d, topk = cfg["L"], cfg["H"], cfg["d"], cfg["topk"]
-    layer = next(iter(correlated_layers(L, H, d, 1, cfg["seed"], device="cpu"))).numpy()
+    c = LONG
+    L, H, d, topk = c["L"], c["H"], c["d"], c["topk"]
     rng = np.random.default_rng(1)
-    rows_per_step = args.ref_rows
+    keys = gaussian_layer(L, 1, d, seed=c["seed"])
+    pool = gaussian_layer(256, H, d, seed=c["seed"] + 1)
+    k_h, ks_h = keys.k.numpy(), keys.k_scale.numpy()
+    qp, qsp, wp = pool.q.numpy(), pool.q_scale.numpy(), pool.w.numpy()
+    nproc = os.cpu_count() or 1
+    rows_per_step = args.ref_rows if args.ref_rows > 0 else nproc
 
     def step():
-        n = 0
-        for t in rng.integers(0, L, size=rows_per_step):
-            O.prefill_rows(layer, topk, [int(t)])
-            n += int(t) + 1
-        return n
+        pos = rng.integers(0, L, size=rows_per_step)
+        pick = rng.integers(0, qp.shape[0], size=rows_per_step)
+        C.prefill_positions(qp[pick], qsp[pick], wp[pick], k_h, ks_h, pos, topk, n_threads=nproc,
+                            want_scores=False)
+        return int((pos + 1).sum())
 
     for _ in range(args.warmup):
         step()
@@ -524,94 +657,31 @@ def run_reference(args, world, rank):
         pairs += step()
     el = time.perf_counter() - t0
     value = pairs / el
+    sample = f"{args.steps} steps x {rows_per_step} uniformly drawn query rows, C++ oracle on {nproc} threads"
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": el * 1e3 / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": "IndexCache prefill stack: 8 layers, L=16384, H=64, d=128, "
-                                   "k=2048, pattern FSFSFSFS (4 indexer layers), rho=0.9 "
-                                   "correlated FP8 E4M3 layers, then the 8x8 top-k overlap",
-                       "sample": f"{rows_per_step} uniformly drawn query rows of an indexer layer per step"},
-            "cpu_baseline": {"value": value, "unit": UNIT, "kind": "oracle", "cores": numpy_threads(),
-                             "sample": f"{args.steps} steps x {rows_per_step} query rows"},
+            "config": {"workload": "200000-token prefill through 47 layers, searched 1/4 IndexCache "
+                                   "pattern (12 indexer layers), H=64, d=128, k=2048, chunks of 8192",
+                       "sample": sample},
+            "cpu_baseline": {"value": value, "unit": UNIT, "kind": "oracle", "cores": nproc,
+                             "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
-    print(json.dumps(line), flush=True)
-
-
-def run_long_prefill_patterns(args, local):
-    """Long-context prefill under several IndexCache patterns: L = 200000, H = 64, d = 128,
-    k = 2048, 47 rho = 0.9 correlated layers, chunks of 8192 queries against the whole causal
-    prefix. Every layer's indexer pass (all 25 chunks) is timed once with CUDA events; an F/S
-    pattern runs exactly its F layers (S layers alias their F buffer: no launch), so its wall
-    time is the sum over its F layers. Prints one JSON line."""
-    from sparse_attention_token_04_b200 import binding as B
-    from synth import SEARCHED_QUARTER_PATTERN, correlated_layers
-
-    device = torch.device("cuda", local)
-    torch.cuda.set_device(device)
-    L, H, d, topk, n_layers, chunk = 200000, 64, 128, 2048, 47, 8192
-    patterns = {
-        "searched 1/4 (12 F)": SEARCHED_QUARTER_PATTERN,
-        "all F (47 F)": "F" * n_layers,
-        "FFFS (36 F)": ("FFFS" * 12)[:n_layers],
-        "FSSS (12 F)": ("FSSS" * 12)[:n_layers],
-    }
-    ws = torch.empty(B.dsa_prefill_workspace_bytes(chunk, H, d, topk), dtype=torch.uint8, device=device)
-    B.dsa_workspace_init(ws)
-    out_idx = torch.empty(chunk, topk, dtype=torch.int32, device=device)
-    stream = torch.cuda.current_stream()
-    layer_ms = []
-    for layer in correlated_layers(L, H, d, n_layers, seed=5, device=device):
-        def one_pass():
-            for c0 in range(0, L, chunk):
-                c1 = min(L, c0 + chunk)
-                B.dsa_indexer_prefill(layer.q[c0:c1], layer.q_scale[c0:c1], layer.w[c0:c1],
-                                      layer.k[:c1], layer.k_scale[:c1], topk, q_pos0=c0,
-                                      out_idx=out_idx[: c1 - c0], want_score=False, workspace=ws)
-        if not layer_ms:
-            one_pass()  # warm-up
-        torch.cuda.synchronize()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        one_pass()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        layer_ms.append(e0.elapsed_time(e1))
-    status = B.dsa_read_device_status(ws)
-    pairs = causal_pairs(L)
-    flops = 2.0 * H * d * pairs
-    peaks, _ = measured_peaks()
-    fp8_peak = FP8_PER_BF16 * float(peaks["bf16_tflops_sustained"])
-    res = {}
-    for name, pat in patterns.items():
-        f_layers = [i for i, c in enumerate(pat) if c == "F"]
-        ms = float(sum(layer_ms[i] for i in f_layers))
-        res[name] = {"f_layers": len(f_layers), "ms": ms,
-                     "speedup_vs_all_f": float(sum(layer_ms)) / ms}
-    mean_ms = float(np.mean(layer_ms))
-    line = {"workload": "long-context prefill: L=200000, H=64, d=128, k=2048, 47 rho=0.9 "
-                        "correlated FP8 layers, chunks of 8192 queries", "device_status": list(status),
-            "per_layer_ms": {"mean": mean_ms, "min": float(min(layer_ms)), "max": float(max(layer_ms))},
-            "per_layer_pairs_per_s": pairs / (mean_ms / 1e3),
-            "per_layer_tflops": flops / (mean_ms / 1e3) / 1e12,
-            "per_layer_frac_fp8": flops / (mean_ms / 1e3) / 1e12 / fp8_peak,
-            "patterns": res}
     print(json.dumps(line), flush=True)
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--e2e-steps", type=int, default=10)
-    ap.add_argument("--decode-steps", type=int, default=50)
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--stack-steps", type=int, default=20)
+    ap.add_argument("--decode-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--ref-rows", type=int, default=8)
-    ap.add_argument("--long-prefill-patterns", action="store_true",
-                    help="time the 200000-token, 47-layer prefill under four F/S patterns instead")
+    ap.add_argument("--ref-rows", type=int, default=0, help="rows per reference step (0: nproc)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("at least 3 warm-up steps")
@@ -621,9 +691,6 @@ def main():
             raise SystemExit("launch N > 1 with torch.distributed.run (one process per GPU)")
     if args.impl == "reference":
         run_reference(args, world, rank)
-        return
-    if args.long_prefill_patterns:
-        run_long_prefill_patterns(args, local)
         return
     try:
         run_ours(args, world, rank, local)

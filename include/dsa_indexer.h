@@ -30,7 +30,9 @@
  *     (env DSA_WAIT_BUDGET_NS, default 2e9 ns per wait).
  *   - A workspace's first DSA_WS_HEADER_BYTES must be zeroed once before first use
  *     (dsa_workspace_init). Calls that share a workspace must not overlap on the GPU.
- *   - Supported shapes: (H, d) in {(8, 64), (64, 128)}, 1 <= topk <= 2048.
+ *   - Supported shapes, per entry point: prefill takes (H, d) in {(8, 64), (64, 128)}; decode
+ *     (and its allocation-free variant) takes only (H, d) = (64, 128) with block_size = 64.
+ *     Every entry point takes 1 <= topk <= 2048. Other shapes return DSA_ERR_UNSUPPORTED.
  */
 #ifndef DSA_INDEXER_H
 #define DSA_INDEXER_H
@@ -113,9 +115,10 @@ DSA_API dsa_status dsa_indexer_prefill(const uint8_t* q, const float* q_scale, c
  *                                                 are not read)
  *   seq_lens      [B]                            i32, 1 <= seq_lens[b] <= max_blocks*block_size
  *   out_idx       [B][topk] i32 logical positions;  out_score [B][topk] f32 or NULL
- * block_size must be 64 and B at most DSA_DECODE_MAX_REQUESTS (else DSA_ERR_UNSUPPORTED, nothing
- * enqueued). A block-table entry outside [0, n_blocks) or a bad length is
- * recorded as DSA_ERR_DEVICE (the request's keys are then read from block 0 / clamped).
+ * Decode is built for H = 64, d = 128 and block_size = 64 only, and for B at most
+ * DSA_DECODE_MAX_REQUESTS; any other shape returns DSA_ERR_UNSUPPORTED with nothing
+ * enqueued. A block-table entry outside [0, n_blocks) or a bad length is recorded as
+ * DSA_ERR_DEVICE (the request's keys are then read from block 0 / clamped).
  * workspace: >= dsa_decode_workspace_bytes(B, max_blocks*block_size, H, d, topk) bytes.
  * -------------------------------------------------------------------------------------*/
 #define DSA_DECODE_MAX_REQUESTS 65535
@@ -145,9 +148,11 @@ DSA_API dsa_status dsa_indexer_decode(const uint8_t* q, const float* q_scale, co
  *   - B must not exceed DSA_NOALLOC_MAX_REQUESTS and B * max_blocks * block_size must not exceed
  *     DSA_NOALLOC_MAX_SCORES; a larger call returns DSA_ERR_UNSUPPORTED and enqueues nothing.
  *     Other errors are those of dsa_indexer_decode.
+ *   - Shapes: as dsa_indexer_decode, i.e. H = 64, d = 128, block_size = 64.
  *   - device_status_out: optional DEVICE int32[2] that receives the call's device-side status
- *     and detail (as dsa_read_device_status reports them); the fixed scratch's status is
- *     cleared at the end of every call, so pass NULL only if those errors are not wanted.
+ *     and detail (as dsa_read_device_status reports them). The fixed scratch's status header
+ *     is cleared on the stream at the start of every call, so each call reports only its own
+ *     device-side errors; pass NULL only if those errors are not wanted.
  *   - The first call on each device looks up the scratch's device address (cudaGetSymbolAddress)
  *     with that device current and caches it; make that first call before any stream capture.
  *   - Every call on a device shares the one scratch array and may leave data in it: calls whose
@@ -230,7 +235,7 @@ DSA_API dsa_status indexcache_run(const char* pattern, int32_t n_layers,
  * out_valid  [1] u64: V = number of non-negative entries of layer 0.
  * out_overlap [n_layers][n_layers] f64 = C / V, or NULL.
  * An entry outside [-1, n_keys) is skipped and recorded as DSA_ERR_DEVICE.
- * workspace: >= DSA_WS_HEADER_BYTES bytes. n_keys <= 1,600,000.
+ * workspace: >= DSA_WS_HEADER_BYTES bytes. n_keys <= 1,500,000 (larger: DSA_ERR_UNSUPPORTED).
  * -------------------------------------------------------------------------------------*/
 DSA_API dsa_status topk_overlap(const int32_t* const* layer_idx, int32_t n_layers, int32_t rows,
                                 int32_t topk, int32_t n_keys, uint64_t* out_counts,

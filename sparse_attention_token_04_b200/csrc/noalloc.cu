@@ -26,8 +26,9 @@ namespace {
 constexpr size_t kScratchBytes =
     decode_layout(DSA_NOALLOC_MAX_REQUESTS, static_cast<size_t>(DSA_NOALLOC_MAX_SCORES)).total;
 
-// Zero at load time; the status header is cleared again at the end of every call, so each call
-// starts with a clean status (the decode launch itself clears the histograms it uses).
+// Zero at load time. Every call clears the status header on its stream before its kernels, so a
+// call reports only its own device-side errors, even after an earlier call that failed part-way
+// (the decode launch itself clears the histograms it uses).
 static __device__ __align__(256) uint8_t g_decode_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
@@ -67,14 +68,14 @@ extern "C" DSA_API dsa_status dsa_indexer_decode_noalloc(
   void* scratch = nullptr;
   dsa_status st = scratch_address(&scratch);
   if (st != DSA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(scratch, 0, DSA_WS_HEADER_BYTES, s) != cudaSuccess) return DSA_ERR_CUDA;
   st = dsa_indexer_decode(q, q_scale, w, k_cache, k_scale_cache, n_blocks, block_size, block_table,
                           max_blocks, seq_lens, B, H, d, topk, out_idx, out_score, scratch,
                           kScratchBytes, stream);
   if (st != DSA_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (device_status_out &&
-      cudaMemcpyAsync(device_status_out, scratch, 2 * sizeof(int32_t), cudaMemcpyDeviceToDevice, s) !=
-          cudaSuccess)
-    return DSA_ERR_CUDA;
-  return cuda_status(cudaMemsetAsync(scratch, 0, DSA_WS_HEADER_BYTES, s));
+  if (device_status_out)
+    return cuda_status(cudaMemcpyAsync(device_status_out, scratch, 2 * sizeof(int32_t),
+                                       cudaMemcpyDeviceToDevice, s));
+  return DSA_OK;
 }

@@ -7,14 +7,16 @@
 // block of QB queries it streams the causal key range in tiles of 128 keys:
 //   warp 0      TMA producer: the block's Q rows (two 256-row B operands) once, then one
 //               [128 keys x d] FP8 K tile per pipeline stage;
-//   warp 1      one thread issues tcgen05.mma kind::f8f6f4 (M = 128 keys, N = 256 =
-//               (256/H) queries x H heads, K = d), FP32 accumulators in TMEM, two
-//               256-column accumulators so the epilogue of one overlaps the MMA of the other;
-//   warps 4-11  two epilogue warpgroups, one per accumulator. Thread = key (its TMEM lane):
-//               it reads the key's H head dot products of each query, applies ReLU, the head
-//               weights, then the query and key scales, masks s > t, and appends the keys it
-//               keeps to its warp's segment of the query's buffer (no atomics: the segment's
-//               count lives in a register of the warp).
+//   warp 1      one thread issues tcgen05.mma kind::f8f6f4 (M = 128 keys, N = queries x H
+//               heads, K = d) into FP32 accumulators in TMEM. The 512 TMEM columns hold four
+//               128-column accumulators in the sample and lean modes and two 256-column ones in
+//               the exact mode, so the epilogue of one overlaps the MMAs of the others;
+//   warps 4..   four epilogue warps per accumulator (16 in the sample and lean modes, 8 in the
+//               exact mode), one per TMEM lane quarter. Thread = key (its TMEM lane): it reads
+//               the key's H head dot products of each query, applies ReLU, the head weights,
+//               then the query and key scales, masks s > t, and appends the keys it keeps to
+//               its warp's segment of the query's buffer (no atomics: the segment's count
+//               lives in a register of the warp).
 //
 // The same kernel runs in three modes:
 //   sample  every S-th key only (a strided tensor map), every valid key appended: a uniform
