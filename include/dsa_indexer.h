@@ -225,6 +225,35 @@ DSA_API dsa_status indexcache_run(const char* pattern, int32_t n_layers,
                                   void* stream);
 
 /* ---------------------------------------------------------------------------------------
+ * Multi-layer-indexer (lagged) variant of indexcache_run ("多层索引器：DeepSeek 稀疏注意力中的重叠
+ * 选择与注意力", abstract: adjacent layers select nearly the same tokens, so a layer can attend the
+ * selection of the previous indexer layer instead of its own; that removes the dependency and
+ * lets every indexer run concurrently with the attention of its layer, and it composes with
+ * IndexCache).
+ *
+ * Arguments as indexcache_run, plus indexer_stream (a second cudaStream_t). Every Full layer's
+ * indexer runs on indexer_stream; `consume` is called for every layer in order and enqueues that
+ * layer's consumer (attention) on `stream`. The buffer layer l's consumer gets is that of the
+ * last Full layer BEFORE l: for a Full layer the previous indexer layer's selection (its own
+ * indexer runs meanwhile), for a Shared layer its source Full layer's (the IndexCache rule).
+ * Layer 0 has no earlier indexer layer and gets its own selection. Before each call of `consume`,
+ * `stream` is made to wait (cudaStreamWaitEvent) for the indexer work that wrote the buffer it
+ * passes; before each Full layer's indexer, indexer_stream waits for all work enqueued on
+ * `stream` so far (the layer's inputs, and every consumer that may still read the buffer about
+ * to be rewritten). When the call returns, `stream` also waits for the last indexer.
+ * 2 <= n_fbufs <= max(2, number of Full layers) (1 is allowed when there is one Full layer):
+ * Full layer m writes f_bufs[m % n_fbufs]; n_fbufs = number of Full layers keeps every layer's
+ * indices. stream and indexer_stream must differ. `consume` may be NULL (then only out_layer_idx is filled).
+ * The workspace is used on indexer_stream only. Errors as indexcache_run.
+ * -------------------------------------------------------------------------------------*/
+DSA_API dsa_status indexcache_run_lagged(const char* pattern, int32_t n_layers,
+                                         const dsa_indexer_shape* shape,
+                                         const dsa_layer_inputs* layers, int32_t* const* f_bufs,
+                                         int32_t n_fbufs, const int32_t** out_layer_idx,
+                                         dsa_after_layer_fn consume, void* user, void* workspace,
+                                         size_t workspace_bytes, void* stream, void* indexer_stream);
+
+/* ---------------------------------------------------------------------------------------
  * Cross-layer top-k overlap ("IndexShare deep-dive report" §1.2: the overlap of layers i
  * and j is |T(i) ∩ T(j)| / k; adjacent layers overlap 70-100% in blocks).
  *
@@ -241,6 +270,53 @@ DSA_API dsa_status topk_overlap(const int32_t* const* layer_idx, int32_t n_layer
                                 int32_t topk, int32_t n_keys, uint64_t* out_counts,
                                 uint64_t* out_valid, double* out_overlap, void* workspace,
                                 size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Exact merge of top-k lists selected over disjoint key ranges of the same rows. The pages
+ * serve one model replica per GPU ("IndexShare deep-dive report" §4.2, Table 1: SGLang with
+ * dp = 8 on one node); they have no counterpart to splitting one request's keys over GPUs.
+ * That split is exact because the top-k of a row ("IndexShare deep-dive report" §1.1) is
+ * contained in the union of the top-k lists of any partition of its keys: each GPU selects
+ * the top-k of its own range (dsa_indexer_decode on its share of the block table), the lists
+ * are gathered, and this call takes the top-k of their union.
+ *   scores     [n_lists][rows][topk] f32   each list row as the indexer writes it: score
+ *   idx        [n_lists][rows][topk] i32   descending, ties by ascending index, -1 / -inf padding
+ *   idx_offset [n_lists][rows] i32 or NULL: added to every valid index of that list row (the
+ *              first key position of the range the list was selected from)
+ *   out_idx    [rows][topk] i32, written; out_score [rows][topk] f32 or NULL
+ * The result is ordered and padded like the indexer's rows, ties going to the lower index. The
+ * lists of one row must hold distinct key positions (disjoint ranges); duplicates are not
+ * removed. 1 <= n_lists <= DSA_MAX_LAYERS, 1 <= topk <= 2048, rows >= 1; outputs must not
+ * alias inputs.
+ * -------------------------------------------------------------------------------------*/
+DSA_API dsa_status dsa_topk_merge(const float* scores, const int32_t* idx, const int32_t* idx_offset,
+                                  int32_t n_lists, int32_t rows, int32_t topk, int32_t* out_idx,
+                                  float* out_score, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Layer-pattern diagnostics from an overlap matrix (host functions; no device work).
+ * "IndexShare deep-dive report" §1.2 / §3.1: the cross-layer overlap of a DSA model forms blocks
+ * of layers whose selections agree, separated by a few transition layers, which uniform F/S
+ * interleaving ignores. §5.2 of the same report: a similarity proxy does not predict model
+ * quality, so these describe an overlap matrix; they do not choose a serving pattern.
+ *
+ * overlap: HOST [n_layers][n_layers] f64 (as topk_overlap writes out_overlap, copied to the host),
+ * 1 <= n_layers <= DSA_MAX_LAYERS.
+ *
+ * dsa_overlap_blocks: block_of_layer[l] (HOST [n_layers] i32) = index of the block of layer l,
+ *   where a new block starts at every layer l > 0 with overlap[l][l-1] < threshold. Returns the
+ *   number of blocks, or -1 for invalid arguments.
+ * dsa_pattern_from_overlap: writes to pattern_out (HOST, n_layers + 1 chars, NUL-terminated) the
+ *   F/S pattern with exactly n_full Full layers, layer 0 Full, that maximises the overlap kept,
+ *   sum_l overlap[l][f(l)] with f(l) the last Full layer at or before l (overlap[l][l] taken as
+ *   1); *retained_out (nullable) = that maximum / n_layers. Exact (dynamic programming); ties go
+ *   to the pattern the recursion meets first. DSA_ERR_INVALID for bad arguments.
+ * -------------------------------------------------------------------------------------*/
+DSA_API int32_t dsa_overlap_blocks(const double* overlap, int32_t n_layers, double threshold,
+                                   int32_t* block_of_layer);
+
+DSA_API dsa_status dsa_pattern_from_overlap(const double* overlap, int32_t n_layers, int32_t n_full,
+                                            char* pattern_out, double* retained_out);
 
 /* ---------------------------------------------------------------------------------------
  * Failure-detection self-test (no counterpart on the pages): launches one CTA that waits,

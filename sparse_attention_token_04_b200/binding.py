@@ -60,9 +60,15 @@ _SIGNATURES = {
     "indexcache_run": (_i32, [ctypes.c_char_p, _i32, ctypes.POINTER(dsa_indexer_shape),
                               ctypes.POINTER(dsa_layer_inputs), ctypes.POINTER(_vp), _i32,
                               ctypes.POINTER(_vp), AFTER_LAYER_FN, _vp, _vp, _sz, _vp]),
+    "indexcache_run_lagged": (_i32, [ctypes.c_char_p, _i32, ctypes.POINTER(dsa_indexer_shape),
+                                     ctypes.POINTER(dsa_layer_inputs), ctypes.POINTER(_vp), _i32,
+                                     ctypes.POINTER(_vp), AFTER_LAYER_FN, _vp, _vp, _sz, _vp, _vp]),
     "topk_overlap": (_i32, [ctypes.POINTER(_vp), _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp,
                             _sz, _vp]),
     "dsa_selftest_wait_timeout": (_i32, [_vp, _sz, _u64, _vp]),
+    "dsa_overlap_blocks": (_i32, [_vp, _i32, ctypes.c_double, _vp]),
+    "dsa_pattern_from_overlap": (_i32, [_vp, _i32, _i32, ctypes.c_char_p, ctypes.POINTER(ctypes.c_double)]),
+    "dsa_topk_merge": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp]),
     "dsa_indexer_decode_noalloc": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _i32, _vp, _i32,
                                           _i32, _i32, _i32, _vp, _vp, _vp, _vp]),
 }
@@ -233,15 +239,8 @@ def dsa_indexcache_workspace_bytes(shape: dsa_indexer_shape) -> int:
     return int(lib().dsa_indexcache_workspace_bytes(ctypes.byref(shape)))
 
 
-def indexcache_run(pattern: str, layers: Sequence[Optional[dict]], topk: int, mode: int = DSA_MODE_PREFILL,
-                   f_bufs: Optional[List[torch.Tensor]] = None, keep_all: bool = True,
-                   q_pos0: int = 0, block_table=None, seq_lens=None,
-                   after_layer: Optional[Callable[[int, int], None]] = None,
-                   workspace=None, stream=None):
-    """IndexCache driver. `layers[l]` is a dict of the layer's tensors (q, q_scale, w, k,
-    k_scale, optional out_score) for prefill, or (q, q_scale, w, k_cache, k_scale_cache) for
-    decode; entries of S layers may be None. Returns (f_bufs, out_layer_ptrs) where
-    out_layer_ptrs[l] is the device address of the buffer holding layer l's indices."""
+def _indexcache_args(pattern, layers, topk, mode, f_bufs, n_bufs_default, q_pos0, block_table,
+                     seq_lens):
     n_layers = len(pattern)
     if len(layers) != n_layers:
         raise ValueError("one layer entry per pattern character")
@@ -262,14 +261,12 @@ def indexcache_run(pattern: str, layers: Sequence[Optional[dict]], topk: int, mo
                               max_blocks=int(block_table.shape[1]), B=B, block_table=block_table,
                               seq_lens=seq_lens)
         rows = B
-    n_full = pattern.count("F")
     if f_bufs is None:
-        n = n_full if keep_all else 1
-        f_bufs = [torch.empty(rows, topk, dtype=torch.int32, device=first["q"].device) for _ in range(n)]
+        f_bufs = [torch.empty(rows, topk, dtype=torch.int32, device=first["q"].device)
+                  for _ in range(n_bufs_default)]
     for b in f_bufs:
         _need(b, "f_buf", torch.int32, (rows, topk))
     arr = (dsa_layer_inputs * n_layers)()
-    keep = []
     for l, lay in enumerate(layers):
         if lay is None:
             continue
@@ -278,15 +275,53 @@ def indexcache_run(pattern: str, layers: Sequence[Optional[dict]], topk: int, mo
         arr[l] = dsa_layer_inputs(lay["q"].data_ptr(), lay["q_scale"].data_ptr(), lay["w"].data_ptr(),
                                   kk.data_ptr(), ks.data_ptr(),
                                   lay["out_score"].data_ptr() if lay.get("out_score") is not None else None)
-        keep.append(lay)
     fb = (_vp * len(f_bufs))(*[b.data_ptr() for b in f_bufs])
-    out_ptrs = (_vp * n_layers)()
+    return shape, arr, fb, f_bufs, first["q"].device
+
+
+def indexcache_run(pattern: str, layers: Sequence[Optional[dict]], topk: int, mode: int = DSA_MODE_PREFILL,
+                   f_bufs: Optional[List[torch.Tensor]] = None, keep_all: bool = True,
+                   q_pos0: int = 0, block_table=None, seq_lens=None,
+                   after_layer: Optional[Callable[[int, int], None]] = None,
+                   workspace=None, stream=None):
+    """IndexCache driver. `layers[l]` is a dict of the layer's tensors (q, q_scale, w, k,
+    k_scale, optional out_score) for prefill, or (q, q_scale, w, k_cache, k_scale_cache) for
+    decode; entries of S layers may be None. Returns (f_bufs, out_layer_ptrs) where
+    out_layer_ptrs[l] is the device address of the buffer holding layer l's indices."""
+    n_full = pattern.count("F")
+    shape, arr, fb, f_bufs, dev = _indexcache_args(pattern, layers, topk, mode, f_bufs,
+                                                   n_full if keep_all else 1, q_pos0, block_table,
+                                                   seq_lens)
+    out_ptrs = (_vp * len(pattern))()
     cb = AFTER_LAYER_FN(lambda l, p, u: after_layer(int(l), int(p or 0))) if after_layer else AFTER_LAYER_FN()
-    nbytes = dsa_indexcache_workspace_bytes(shape)
-    ws = _workspace(nbytes, first["q"].device, workspace, stream)
-    _check(lib().indexcache_run(pattern.encode(), n_layers, ctypes.byref(shape), arr, fb, len(f_bufs),
+    ws = _workspace(dsa_indexcache_workspace_bytes(shape), dev, workspace, stream)
+    _check(lib().indexcache_run(pattern.encode(), len(pattern), ctypes.byref(shape), arr, fb, len(f_bufs),
                                 out_ptrs, cb, None, _ptr(ws), ws.numel(), _stream(stream)),
            "indexcache_run")
+    return f_bufs, [int(p or 0) for p in out_ptrs]
+
+
+def indexcache_run_lagged(pattern: str, layers: Sequence[Optional[dict]], topk: int,
+                          indexer_stream, mode: int = DSA_MODE_PREFILL,
+                          f_bufs: Optional[List[torch.Tensor]] = None, keep_all: bool = True,
+                          q_pos0: int = 0, block_table=None, seq_lens=None,
+                          consume: Optional[Callable[[int, int], None]] = None,
+                          workspace=None, stream=None):
+    """Multi-layer-indexer variant of indexcache_run: every Full layer's indexer runs on
+    `indexer_stream` while layer l's consumer (called as consume(l, ptr), enqueuing on `stream`)
+    reads the selection of the last Full layer before l (layer 0: its own). Returns (f_bufs,
+    out_layer_ptrs)."""
+    n_full = pattern.count("F")
+    shape, arr, fb, f_bufs, dev = _indexcache_args(pattern, layers, topk, mode, f_bufs,
+                                                   n_full if keep_all else min(2, n_full), q_pos0,
+                                                   block_table, seq_lens)
+    out_ptrs = (_vp * len(pattern))()
+    cb = AFTER_LAYER_FN(lambda l, p, u: consume(int(l), int(p or 0))) if consume else AFTER_LAYER_FN()
+    ws = _workspace(dsa_indexcache_workspace_bytes(shape), dev, workspace, stream)
+    _check(lib().indexcache_run_lagged(pattern.encode(), len(pattern), ctypes.byref(shape), arr, fb,
+                                       len(f_bufs), out_ptrs, cb, None, _ptr(ws), ws.numel(),
+                                       _stream(stream), _stream(indexer_stream)),
+           "indexcache_run_lagged")
     return f_bufs, [int(p or 0) for p in out_ptrs]
 
 
@@ -327,6 +362,60 @@ def topk_overlap_ptrs(ptrs: Sequence[int], rows: int, topk: int, n_keys: int, ou
 def dsa_selftest_wait_timeout(workspace: torch.Tensor, budget_ns: int, stream=None) -> None:
     _check(lib().dsa_selftest_wait_timeout(_ptr(workspace), workspace.numel(), int(budget_ns),
                                            _stream(stream)), "dsa_selftest_wait_timeout")
+
+
+def dsa_topk_merge(scores, idx, idx_offset=None, out_idx=None, out_score=None, stream=None):
+    """Top-k of the union of n_lists top-k lists per row: scores [n_lists][rows][topk] f32 and
+    idx [n_lists][rows][topk] i32 (each row sorted as the indexer writes it), idx_offset
+    [n_lists][rows] i32 added to each list row's valid indices (or None) -> (out_idx[rows][topk]
+    i32, out_score[rows][topk] f32)."""
+    n_lists, rows, topk = (int(x) for x in idx.shape)
+    _need(idx, "idx", torch.int32)
+    _need(scores, "scores", torch.float32, (n_lists, rows, topk))
+    if idx_offset is not None:
+        _need(idx_offset, "idx_offset", torch.int32, (n_lists, rows))
+    if out_idx is None:
+        out_idx = torch.empty(rows, topk, dtype=torch.int32, device=idx.device)
+    _need(out_idx, "out_idx", torch.int32, (rows, topk))
+    if out_score is None:
+        out_score = torch.empty(rows, topk, dtype=torch.float32, device=idx.device)
+    _need(out_score, "out_score", torch.float32, (rows, topk))
+    _check(lib().dsa_topk_merge(_ptr(scores), _ptr(idx), _ptr(idx_offset), n_lists, rows, topk,
+                                _ptr(out_idx), _ptr(out_score), _stream(stream)), "dsa_topk_merge")
+    return out_idx, out_score
+
+
+def _host_overlap(overlap):
+    import numpy as np
+    o = np.ascontiguousarray(np.asarray(overlap.cpu() if isinstance(overlap, torch.Tensor) else overlap,
+                                        dtype=np.float64))
+    if o.ndim != 2 or o.shape[0] != o.shape[1]:
+        raise ValueError("overlap must be a square [n_layers][n_layers] matrix")
+    return o
+
+
+def dsa_overlap_blocks(overlap, threshold: float):
+    """Blocks of layers from an overlap matrix (host): returns (n_blocks, block_of_layer list)."""
+    import numpy as np
+    o = _host_overlap(overlap)
+    n = o.shape[0]
+    out = np.zeros(n, dtype=np.int32)
+    nb = int(lib().dsa_overlap_blocks(o.ctypes.data, n, float(threshold), out.ctypes.data))
+    if nb < 0:
+        raise DsaError(DSA_ERR_INVALID, "dsa_overlap_blocks")
+    return nb, out.tolist()
+
+
+def dsa_pattern_from_overlap(overlap, n_full: int):
+    """The F/S pattern with n_full Full layers that keeps the most overlap (host): returns
+    (pattern, mean overlap kept per layer)."""
+    o = _host_overlap(overlap)
+    n = o.shape[0]
+    buf = ctypes.create_string_buffer(n + 1)
+    kept = ctypes.c_double(0.0)
+    _check(lib().dsa_pattern_from_overlap(o.ctypes.data, n, int(n_full), buf, ctypes.byref(kept)),
+           "dsa_pattern_from_overlap")
+    return buf.value.decode(), float(kept.value)
 
 
 DSA_DECODE_MAX_REQUESTS = 65535

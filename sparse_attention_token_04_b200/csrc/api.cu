@@ -185,25 +185,21 @@ DSA_API size_t dsa_indexcache_workspace_bytes(const dsa_indexer_shape* shape) {
   return 0;
 }
 
-DSA_API dsa_status indexcache_run(const char* pattern, int32_t n_layers,
-                                  const dsa_indexer_shape* shape, const dsa_layer_inputs* layers,
-                                  int32_t* const* f_bufs, int32_t n_fbufs,
-                                  const int32_t** out_layer_idx, dsa_after_layer_fn after_layer,
-                                  void* user, void* workspace, size_t workspace_bytes,
-                                  void* stream) {
+// Validates an IndexCache call (pattern, buffers, every Full layer's inputs, workspace) before
+// anything is enqueued; returns the number of Full layers in *n_full.
+static dsa_status check_indexcache(const char* pattern, int32_t n_layers,
+                                   const dsa_indexer_shape* shape, const dsa_layer_inputs* layers,
+                                   int32_t* const* f_bufs, const int32_t** out_layer_idx,
+                                   void* workspace, size_t workspace_bytes, int* n_full) {
   if (!pattern || !shape || !layers || !f_bufs || !out_layer_idx || n_layers < 1) return DSA_ERR_INVALID;
   if (static_cast<int64_t>(std::strlen(pattern)) != n_layers) return DSA_ERR_INVALID;
-  int n_full = 0;
+  *n_full = 0;
   for (int l = 0; l < n_layers; ++l) {
-    if (pattern[l] == 'F') ++n_full;
+    if (pattern[l] == 'F') ++*n_full;
     else if (pattern[l] != 'S') return DSA_ERR_INVALID;
   }
   if (pattern[0] != 'F') return DSA_ERR_INVALID;  // the first layer is always Full
-  if (n_fbufs != 1 && n_fbufs != n_full) return DSA_ERR_INVALID;
-  for (int m = 0; m < n_fbufs; ++m)
-    if (!f_bufs[m]) return DSA_ERR_INVALID;
   if (shape->mode != DSA_MODE_PREFILL && shape->mode != DSA_MODE_DECODE) return DSA_ERR_INVALID;
-  // Validate every Full layer before anything is enqueued.
   for (int l = 0; l < n_layers; ++l) {
     if (pattern[l] != 'F') continue;
     const dsa_layer_inputs& in = layers[l];
@@ -219,6 +215,36 @@ DSA_API dsa_status indexcache_run(const char* pattern, int32_t n_layers,
   }
   const size_t need = dsa_indexcache_workspace_bytes(shape);
   if (!workspace || need == 0 || workspace_bytes < need || !aligned(workspace, 256)) return DSA_ERR_INVALID;
+  return DSA_OK;
+}
+
+// One Full layer's indexer into buf on stream.
+static dsa_status run_full_layer(const dsa_indexer_shape* shape, const dsa_layer_inputs& in,
+                                 int32_t* buf, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
+  if (shape->mode == DSA_MODE_PREFILL)
+    return dsa_indexer_prefill(in.q, in.q_scale, in.w, in.k, in.k_scale, shape->Lk, shape->q_pos0,
+                               shape->Lq, shape->H, shape->d, shape->topk, buf, in.out_score,
+                               workspace, workspace_bytes, stream);
+  return dsa_indexer_decode(in.q, in.q_scale, in.w, in.k, in.k_scale, shape->n_blocks,
+                            shape->block_size, shape->block_table, shape->max_blocks,
+                            shape->seq_lens, shape->B, shape->H, shape->d, shape->topk, buf,
+                            in.out_score, workspace, workspace_bytes, stream);
+}
+
+DSA_API dsa_status indexcache_run(const char* pattern, int32_t n_layers,
+                                  const dsa_indexer_shape* shape, const dsa_layer_inputs* layers,
+                                  int32_t* const* f_bufs, int32_t n_fbufs,
+                                  const int32_t** out_layer_idx, dsa_after_layer_fn after_layer,
+                                  void* user, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  int n_full = 0;
+  dsa_status st = check_indexcache(pattern, n_layers, shape, layers, f_bufs, out_layer_idx,
+                                   workspace, workspace_bytes, &n_full);
+  if (st != DSA_OK) return st;
+  if (n_fbufs != 1 && n_fbufs != n_full) return DSA_ERR_INVALID;
+  for (int m = 0; m < n_fbufs; ++m)
+    if (!f_bufs[m]) return DSA_ERR_INVALID;
 
   int m = 0;
   const int32_t* cached = nullptr;
@@ -226,24 +252,75 @@ DSA_API dsa_status indexcache_run(const char* pattern, int32_t n_layers,
     if (pattern[l] == 'F') {
       int32_t* buf = f_bufs[n_fbufs == 1 ? 0 : m];
       ++m;
-      const dsa_layer_inputs& in = layers[l];
-      dsa_status st;
-      if (shape->mode == DSA_MODE_PREFILL)
-        st = dsa_indexer_prefill(in.q, in.q_scale, in.w, in.k, in.k_scale, shape->Lk, shape->q_pos0,
-                                 shape->Lq, shape->H, shape->d, shape->topk, buf, in.out_score,
-                                 workspace, workspace_bytes, stream);
-      else
-        st = dsa_indexer_decode(in.q, in.q_scale, in.w, in.k, in.k_scale, shape->n_blocks,
-                                shape->block_size, shape->block_table, shape->max_blocks,
-                                shape->seq_lens, shape->B, shape->H, shape->d, shape->topk, buf,
-                                in.out_score, workspace, workspace_bytes, stream);
-      if (st != DSA_OK) return st;
+      if ((st = run_full_layer(shape, layers[l], buf, workspace, workspace_bytes, stream)) != DSA_OK)
+        return st;
       cached = buf;
     }
     out_layer_idx[l] = cached;  // an S layer reads T_f(l): the buffer of the last F layer
     if (after_layer) after_layer(l, cached, user);
   }
   return DSA_OK;
+}
+
+DSA_API dsa_status indexcache_run_lagged(const char* pattern, int32_t n_layers,
+                                         const dsa_indexer_shape* shape,
+                                         const dsa_layer_inputs* layers, int32_t* const* f_bufs,
+                                         int32_t n_fbufs, const int32_t** out_layer_idx,
+                                         dsa_after_layer_fn consume, void* user, void* workspace,
+                                         size_t workspace_bytes, void* stream,
+                                         void* indexer_stream) {
+  int n_full = 0;
+  dsa_status st = check_indexcache(pattern, n_layers, shape, layers, f_bufs, out_layer_idx,
+                                   workspace, workspace_bytes, &n_full);
+  if (st != DSA_OK) return st;
+  // A Full layer's consumer reads the previous Full layer's buffer while the layer's own
+  // indexer writes: two buffers at least (one suffices for a single Full layer).
+  const int min_bufs = n_full >= 2 ? 2 : 1;
+  if (n_fbufs < min_bufs || n_fbufs > (n_full > 2 ? n_full : 2)) return DSA_ERR_INVALID;
+  for (int m = 0; m < n_fbufs; ++m)
+    if (!f_bufs[m]) return DSA_ERR_INVALID;
+  if (stream == indexer_stream) return DSA_ERR_INVALID;  // the point is two streams
+  cudaStream_t main_s = static_cast<cudaStream_t>(stream);
+  cudaStream_t idx_s = static_cast<cudaStream_t>(indexer_stream);
+
+  // One completion event per Full layer (the indexer's work on indexer_stream) and one event
+  // marking where each Full layer's inputs are ready on the consumer stream.
+  const int n_events = n_full + 1;
+  cudaEvent_t* ev = new cudaEvent_t[n_events];
+  int made = 0;
+  for (; made < n_events; ++made)
+    if (cudaEventCreateWithFlags(&ev[made], cudaEventDisableTiming) != cudaSuccess) break;
+  auto cleanup = [&](dsa_status s) {
+    for (int i = 0; i < made; ++i) cudaEventDestroy(ev[i]);  // released once they complete
+    delete[] ev;
+    return s;
+  };
+  if (made < n_events) return cleanup(DSA_ERR_CUDA);
+  cudaEvent_t ready = ev[n_full];
+
+  int m = -1;  // index of the last Full layer so far
+  for (int l = 0; l < n_layers; ++l) {
+    int src;
+    if (pattern[l] == 'F') {
+      ++m;
+      // Everything enqueued on the consumer stream so far (the layer's inputs; every consumer
+      // that may still read the buffer about to be rewritten) precedes this indexer.
+      if (cudaEventRecord(ready, main_s) != cudaSuccess || cudaStreamWaitEvent(idx_s, ready, 0) != cudaSuccess)
+        return cleanup(DSA_ERR_CUDA);
+      if ((st = run_full_layer(shape, layers[l], f_bufs[m % n_fbufs], workspace, workspace_bytes,
+                               idx_s)) != DSA_OK)
+        return cleanup(st);
+      if (cudaEventRecord(ev[m], idx_s) != cudaSuccess) return cleanup(DSA_ERR_CUDA);
+      src = (m == 0) ? 0 : m - 1;  // the previous indexer layer; layer 0 has only its own
+    } else {
+      src = m;  // the source Full layer, whose indexer ran during that layer's consumer
+    }
+    if (cudaStreamWaitEvent(main_s, ev[src], 0) != cudaSuccess) return cleanup(DSA_ERR_CUDA);
+    out_layer_idx[l] = f_bufs[src % n_fbufs];
+    if (consume) consume(l, out_layer_idx[l], user);
+  }
+  if (cudaStreamWaitEvent(main_s, ev[m], 0) != cudaSuccess) return cleanup(DSA_ERR_CUDA);
+  return cleanup(DSA_OK);
 }
 
 DSA_API dsa_status topk_overlap(const int32_t* const* layer_idx, int32_t n_layers, int32_t rows,
@@ -261,6 +338,16 @@ DSA_API dsa_status topk_overlap(const int32_t* const* layer_idx, int32_t n_layer
   if (sms < 1) return DSA_ERR_CUDA;
   return launch_overlap(layer_idx, n_layers, rows, topk, n_keys, out_counts, out_valid, out_overlap,
                         workspace, static_cast<cudaStream_t>(stream), sms);
+}
+
+DSA_API dsa_status dsa_topk_merge(const float* scores, const int32_t* idx, const int32_t* idx_offset,
+                                  int32_t n_lists, int32_t rows, int32_t topk, int32_t* out_idx,
+                                  float* out_score, void* stream) {
+  if (!scores || !idx || !out_idx) return DSA_ERR_INVALID;
+  if (n_lists < 1 || n_lists > DSA_MAX_LAYERS || rows < 1 || topk < 1) return DSA_ERR_INVALID;
+  if (topk > DSA_MAX_TOPK) return DSA_ERR_UNSUPPORTED;
+  return launch_topk_merge(scores, idx, idx_offset, n_lists, rows, topk, out_idx, out_score,
+                           static_cast<cudaStream_t>(stream));
 }
 
 DSA_API dsa_status dsa_selftest_wait_timeout(void* workspace, size_t workspace_bytes,

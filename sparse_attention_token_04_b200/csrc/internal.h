@@ -133,6 +133,10 @@ dsa_status launch_overlap(const int32_t* const* layer_idx, int32_t n_layers, int
                           int32_t topk, int32_t n_keys, uint64_t* out_counts, uint64_t* out_valid,
                           double* out_overlap, void* ws, cudaStream_t stream, int num_sms);
 dsa_status launch_selftest_wait(void* ws, uint64_t budget_ns, cudaStream_t stream);
+// Top-k of the union of n_lists sorted top-k lists per row (dsa_topk_merge).
+dsa_status launch_topk_merge(const float* scores, const int32_t* idx, const int32_t* offsets,
+                             int n_lists, int rows, int topk, int32_t* out_idx, float* out_score,
+                             cudaStream_t stream);
 
 // Tensor-map encoding through the driver entry point (no link-time libcuda dependency).
 // Rows of row_bytes bytes, row_stride bytes apart (0: packed), boxes of box_rows rows.
