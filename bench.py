@@ -495,6 +495,78 @@ def run_decode(args, world, rank, device, peaks):
             "gpu_launches": 3 * n_full * args.decode_steps}
 
 
+def run_mli_decode(args, world, rank, device):
+    """The 47-layer decode step with a consumer on every layer, under plain IndexCache and under
+    the lagged multi-layer-indexer mode at the same retention (searched 1/4 pattern). The consumer
+    stands in for the model's sparse attention: it gathers every request's selected rows of a
+    576-wide bf16 latent cache (one cache shared by all layers) and runs softmax(q K^T) V for 128
+    query heads with PyTorch ops on the consumer stream. Plain: each layer's consumer follows its
+    own indexer on one stream. Lagged: every Full layer's indexer runs on a second stream while
+    the consumers read the previous indexer layer's selection."""
+    from sparse_attention_token_04_b200 import binding as B
+    from synth import SEARCHED_QUARTER_PATTERN, decode_lengths, paged_decode_layers
+
+    cfg = DECODE
+    seed = rank_seed(cfg["seed"], rank)
+    lens = decode_lengths(cfg["B"], cfg["lo"], cfg["hi"], seed)
+    table, seq, gen = paged_decode_layers(lens, cfg["H"], cfg["d"], cfg["n_layers"], seed, device=device)
+    pattern = SEARCHED_QUARTER_PATTERN
+    layers = [lay if pattern[l] == "F" else None for l, lay in enumerate(gen)]
+    inputs = [None if l is None else {"q": l.q, "q_scale": l.q_scale, "w": l.w, "k_cache": l.k_cache,
+                                      "k_scale_cache": l.k_scale_cache} for l in layers]
+    topk, Bn, heads, dkv, dv = cfg["topk"], cfg["B"], 128, 576, 512
+    n_slots = int(layers[0].k_cache.shape[0]) * 64
+    g = torch.Generator(device=device)
+    g.manual_seed(seed + 7)
+    latent = torch.randn(n_slots, dkv, generator=g, device=device).to(torch.bfloat16)
+    q_att = torch.randn(Bn, heads, dkv, generator=g, device=device).to(torch.bfloat16)
+    scale = 1.0 / math.sqrt(dkv)
+    bufs = [torch.empty(Bn, topk, dtype=torch.int32, device=device) for _ in range(2)]
+    by_ptr = {b.data_ptr(): b for b in bufs}
+    ws = torch.empty(B.dsa_decode_workspace_bytes(Bn, table.shape[1] * 64, cfg["H"], cfg["d"], topk),
+                     dtype=torch.uint8, device=device)
+    B.dsa_workspace_init(ws)
+    side = torch.cuda.Stream(device=device)
+    stream = torch.cuda.current_stream()
+
+    def consume(l, ptr):
+        idx = by_ptr[ptr].long()
+        valid = idx >= 0
+        phys = table.long().gather(1, (idx.clamp(min=0) // 64)) * 64 + idx.clamp(min=0) % 64
+        kv = latent.index_select(0, phys.view(-1)).view(Bn, topk, dkv)
+        sc = torch.bmm(q_att, kv.transpose(1, 2)).float() * scale
+        sc.masked_fill_(~valid[:, None, :], float("-inf"))
+        torch.bmm(torch.softmax(sc, dim=-1).to(torch.bfloat16), kv[..., :dv])
+
+    def plain():
+        B.indexcache_run(pattern, inputs, topk, mode=B.DSA_MODE_DECODE, f_bufs=bufs[:1],
+                         block_table=table, seq_lens=seq, workspace=ws, after_layer=consume)
+
+    def lagged():
+        B.indexcache_run_lagged(pattern, inputs, topk, side, mode=B.DSA_MODE_DECODE, f_bufs=bufs,
+                                block_table=table, seq_lens=seq, workspace=ws, consume=consume)
+
+    def consumers_only():
+        for l in range(len(pattern)):
+            consume(l, bufs[0].data_ptr())
+
+    res = {}
+    for name, fn in (("plain", plain), ("lagged", lagged), ("consumers_only", consumers_only)):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        res[name] = timed(stream, fn, args.mli_steps) / args.mli_steps
+    if B.dsa_read_device_status(ws) != (0, 0):
+        raise RuntimeError("device status after the lagged decode steps")
+    return {"workload": "47-layer decode step, 32 requests U[10000,200000], searched 1/4 pattern (12 "
+                        "indexer layers), a sparse-attention stand-in consumer on every layer (gather of "
+                        "the 2048 selected rows of a 576-wide bf16 latent cache, softmax(qK^T)V for 128 "
+                        "heads, PyTorch ops)",
+            "plain_indexcache_ms": res["plain"], "lagged_mli_ms": res["lagged"],
+            "consumers_alone_ms": res["consumers_only"],
+            "speedup_lagged_vs_plain": res["plain"] / res["lagged"], "steps": args.mli_steps}
+
+
 # DRAM bytes (read + write) per cached key of decode_indexer_kernel from one ncu capture of this
 # workload, or None when the kernel changed after the capture.
 DECODE_SCORING_DRAM_BYTES_PER_KEY = 5.034e8 / 3737801
@@ -588,6 +660,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.empty_cache()
     stack = run_stack16k(args, world, rank, device, peaks, peak_kind) if args.stack_steps > 0 else None
     decode = run_decode(args, world, rank, device, peaks) if args.decode_steps > 0 else None
+    mli = run_mli_decode(args, world, rank, device) if args.mli_steps > 0 else None
 
     if rank == 0:
         c = LONG
@@ -614,6 +687,7 @@ def run_ours(args, world, rank, local):
             "e2e": long["e2e"],
             "stack_16k": stack,
             "decode": decode,
+            "mli_decode": mli,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
@@ -680,6 +754,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--stack-steps", type=int, default=20)
     ap.add_argument("--decode-steps", type=int, default=20)
+    ap.add_argument("--mli-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-rows", type=int, default=0, help="rows per reference step (0: nproc)")
     args = ap.parse_args()

@@ -35,6 +35,7 @@
 // max(D, 0) = 2^25 * sat(D * 2^-25) exactly (power-of-two scalings, no clipping at 1), and
 // the 2^25 is folded into the stored head weights.
 #include <cstddef>
+#include <type_traits>
 
 #include "common.cuh"
 #include "internal.h"
@@ -171,6 +172,137 @@ __device__ __noinline__ void cut_back(uint64_t* buf, uint32_t seg_stride, uint32
   if (rank < 4) wcnt[rank] = (kept + 3u - rank) >> 2;
   if (rank == 0 && T != 0) *thr = T;
   gs.sync();
+}
+
+// The head-weighted ReLU sums of one epilogue thread's key for the QPW queries of its
+// accumulator: reads QPW * H TMEM columns in 32-column chunks (double-buffered tcgen05.ld)
+// and returns, per query, sum_j w'[j] * sat(D_j * 2^-25) with w' = 2^25 w (stored so in wq).
+template <int H, int QPW>
+__device__ __forceinline__ void head_sums(uint32_t taddr0, const float (*wq)[H], float (&out)[QPW]) {
+  constexpr int NCH = QPW * H / 32;
+  uint32_t ra[32], rb[32];
+  tmem_ld_32x32b_x32(taddr0, ra);
+  tmem_wait_ld_regs(ra);
+  if constexpr (H == 64) {
+    // 64 heads per query: packed FMA over head pairs, four float2 partial sums per query.
+    float2 acc[QPW][4];
+#pragma unroll
+    for (int qi = 0; qi < QPW; ++qi)
+#pragma unroll
+      for (int a = 0; a < 4; ++a) acc[qi][a] = make_float2(0.0f, 0.0f);
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      uint32_t(&cur)[32] = (c & 1) ? rb : ra;
+      uint32_t(&nxt)[32] = (c & 1) ? ra : rb;
+      if (c + 1 < NCH) tmem_ld_32x32b_x32(taddr0 + (c + 1) * 32, nxt);
+      const int qi = c >> 1;
+#pragma unroll
+      for (int j = 0; j < 32; j += 4) {
+        const int h = (c & 1) * 32 + j;
+        const float4 wv = *reinterpret_cast<const float4*>(&wq[qi][h]);
+        const float r0 = __saturatef(__uint_as_float(cur[j + 0]) * 0x1p-25f);
+        const float r1 = __saturatef(__uint_as_float(cur[j + 1]) * 0x1p-25f);
+        const float r2 = __saturatef(__uint_as_float(cur[j + 2]) * 0x1p-25f);
+        const float r3 = __saturatef(__uint_as_float(cur[j + 3]) * 0x1p-25f);
+        const int a = QPW >= 4 ? ((j >> 2) & 1) * 2 : 0;  // fewer chains when registers are scarce
+        acc[qi][a] = __ffma2_rn(make_float2(wv.x, wv.y), make_float2(r0, r1), acc[qi][a]);
+        acc[qi][a + 1] = __ffma2_rn(make_float2(wv.z, wv.w), make_float2(r2, r3), acc[qi][a + 1]);
+      }
+      if (c + 1 < NCH) tmem_wait_ld_regs(nxt);
+    }
+#pragma unroll
+    for (int qi = 0; qi < QPW; ++qi)
+      out[qi] = ((acc[qi][0].x + acc[qi][0].y) + (acc[qi][1].x + acc[qi][1].y)) +
+                ((acc[qi][2].x + acc[qi][2].y) + (acc[qi][3].x + acc[qi][3].y));
+  } else {
+    // 8 heads per query: one scalar chain per query, four queries per chunk.
+#pragma unroll
+    for (int qi = 0; qi < QPW; ++qi) out[qi] = 0.0f;
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      uint32_t(&cur)[32] = (c & 1) ? rb : ra;
+      uint32_t(&nxt)[32] = (c & 1) ? ra : rb;
+      if (c + 1 < NCH) tmem_ld_32x32b_x32(taddr0 + (c + 1) * 32, nxt);
+#pragma unroll
+      for (int j = 0; j < 32; j += 4) {
+        const int col = c * 32 + j;
+        const int qi = col / H, h = col % H;
+        const float4 wv = *reinterpret_cast<const float4*>(&wq[qi][h]);
+        out[qi] = fmaf(wv.x, __saturatef(__uint_as_float(cur[j + 0]) * 0x1p-25f), out[qi]);
+        out[qi] = fmaf(wv.y, __saturatef(__uint_as_float(cur[j + 1]) * 0x1p-25f), out[qi]);
+        out[qi] = fmaf(wv.z, __saturatef(__uint_as_float(cur[j + 2]) * 0x1p-25f), out[qi]);
+        out[qi] = fmaf(wv.w, __saturatef(__uint_as_float(cur[j + 3]) * 0x1p-25f), out[qi]);
+      }
+      if (c + 1 < NCH) tmem_wait_ld_regs(nxt);
+    }
+  }
+}
+
+// Sample and lean passes, H = 64, two queries per accumulator: the head sums read with the 16x256b TMEM
+// shape. Thread t = 4g + i of the warp holds, of its lane quarter, lanes g, g+8, g+16, g+24
+// (lane slot ls = lane / 8) and of each query the 16 heads 8m+2i, 8m+2i+1 (m = 0..7), so it needs
+// only those 32 head weights per tile instead of all 128: the weights' broadcast loads, which
+// kept the load/store unit's register writeback about three quarters busy in the 32x32b form,
+// shrink fourfold. wq holds each query's weights
+// permuted to [i][m][2] (wq[q][16 i + 2 m + e] = w'[q][8 m + 2 i + e]), so a thread's eight
+// weights of a 32-column half are two 16-byte loads, reused for both lane halves. Returns in s
+// the thread's partial sums: s[ls][q] over its 16 heads of query q.
+__device__ __forceinline__ void lean_partials(uint32_t taddr0, const float* wq, uint32_t i,
+                                              float (&s)[4][2]) {
+  float2 acc[4][2];
+#pragma unroll
+  for (int ls = 0; ls < 4; ++ls)
+#pragma unroll
+    for (int q = 0; q < 2; ++q) acc[ls][q] = make_float2(0.0f, 0.0f);
+  // Eight loads of 16 lanes x 32 columns, step k = 4 q + 2 cc + h: query q, column half cc,
+  // lane half h (h fastest, so a weight octet serves two loads).
+  auto addr = [&](int k) {
+    return taddr0 + (static_cast<uint32_t>((k & 1) * 16) << 16) + (k >> 2) * 64 + ((k >> 1) & 1) * 32;
+  };
+  uint32_t ra[16], rb[16];
+  float wv[8];
+  tmem_ld_16x256b_x4(addr(0), ra);
+  tmem_wait_ld_regs16(ra);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    uint32_t(&cur)[16] = (k & 1) ? rb : ra;
+    uint32_t(&nxt)[16] = (k & 1) ? ra : rb;
+    if (k + 1 < 8) tmem_ld_16x256b_x4(addr(k + 1), nxt);
+    const int q = k >> 2, cc = (k >> 1) & 1, h = k & 1;
+    if (h == 0) {
+      const float4 w0 = *reinterpret_cast<const float4*>(wq + q * 64 + i * 16 + cc * 8);
+      const float4 w1 = *reinterpret_cast<const float4*>(wq + q * 64 + i * 16 + cc * 8 + 4);
+      wv[0] = w0.x; wv[1] = w0.y; wv[2] = w0.z; wv[3] = w0.w;
+      wv[4] = w1.x; wv[5] = w1.y; wv[6] = w1.z; wv[7] = w1.w;
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const float2 w = make_float2(wv[2 * m], wv[2 * m + 1]);
+      const float r0 = __saturatef(__uint_as_float(cur[4 * m + 0]) * 0x1p-25f);
+      const float r1 = __saturatef(__uint_as_float(cur[4 * m + 1]) * 0x1p-25f);
+      const float r2 = __saturatef(__uint_as_float(cur[4 * m + 2]) * 0x1p-25f);
+      const float r3 = __saturatef(__uint_as_float(cur[4 * m + 3]) * 0x1p-25f);
+      acc[2 * h][q] = __ffma2_rn(w, make_float2(r0, r1), acc[2 * h][q]);
+      acc[2 * h + 1][q] = __ffma2_rn(w, make_float2(r2, r3), acc[2 * h + 1][q]);
+    }
+    if (k + 1 < 8) tmem_wait_ld_regs16(nxt);
+  }
+#pragma unroll
+  for (int ls = 0; ls < 4; ++ls)
+#pragma unroll
+    for (int q = 0; q < 2; ++q) s[ls][q] = acc[ls][q].x + acc[ls][q].y;
+}
+
+// Sum of the four partials of lane slot i over the four threads 4g..4g+3 (reduce-scatter over
+// xor partners 2 and 1): returns, in every thread, the full sum of its own lane slot i.
+__device__ __forceinline__ float slot_total(const float (&s)[4], uint32_t i) {
+  const bool hi = (i & 2u) != 0, lo = (i & 1u) != 0;
+  const float send_a = hi ? s[0] : s[2], send_b = hi ? s[1] : s[3];
+  const float keep_a = hi ? s[2] : s[0], keep_b = hi ? s[3] : s[1];
+  const float u0 = keep_a + __shfl_xor_sync(0xFFFFFFFFu, send_a, 2);
+  const float u1 = keep_b + __shfl_xor_sync(0xFFFFFFFFu, send_b, 2);
+  const float send = lo ? u0 : u1, keep = lo ? u1 : u0;
+  return keep + __shfl_xor_sync(0xFFFFFFFFu, send, 1);
 }
 
 template <int H, int D, int MODE>
@@ -340,8 +472,10 @@ __global__ void __launch_bounds__(PRoles<H, MODE>::THREADS, 1)
       const int row_base = qb * C::QB + qbase;
       for (int i = rank; i < QPW * H; i += 128) {
         const int qi = i / H, j = i % H, row = row_base + qi;
-        sm.wq[qbase + qi][j] = (row < p.Lq) ? __ldg(&p.w[static_cast<size_t>(row) * H + j]) * 0x1p25f
-                                            : 0.0f;
+        // the sample and lean passes with H = 64 read their weights permuted (see lean_partials)
+        const int slot = (MODE != kModeExact && H == 64) ? ((j & 7) >> 1) * 16 + (j >> 3) * 2 + (j & 1) : j;
+        sm.wq[qbase + qi][slot] = (row < p.Lq) ? __ldg(&p.w[static_cast<size_t>(row) * H + j]) * 0x1p25f
+                                               : 0.0f;
       }
       for (int qi = rank; qi < QPW; qi += 128) {
         const int row = row_base + qi;
@@ -354,12 +488,74 @@ __global__ void __launch_bounds__(PRoles<H, MODE>::THREADS, 1)
 #pragma unroll
       for (int qi = 0; qi < QPW; ++qi) cw[qi] = 0u;
       const int nt = ntiles_of(qb);
-      int v = static_cast<int>(wl * 32u + lane);  // this thread's row of the key tensor map
+      // This thread's key (row of the key tensor map): its TMEM lane, or in the sample and lean
+      // passes with H = 64 the lane slot the head-sum reduction leaves with it (lane g + 8 i,
+      // t = 4 g + i).
+      const uint32_t key_lane = (MODE != kModeExact && H == 64) ? (lane >> 2) + 8u * (lane & 3u) : lane;
+      int v = static_cast<int>(wl * 32u + key_lane);
       auto scale_of = [&](int vi) {
         return vi < p.nkeys ? __ldg(&p.k_scale[static_cast<size_t>(vi) * p.stride]) : 0.0f;
       };
       float sk_next = scale_of(v);
       bool good = true;
+      if constexpr (MODE != kModeExact && H == 64) {
+        // Per query of this warp, in registers: the threshold T as (score, largest key index
+        // taken at that score) and the query scale; the queries' segments are one row pitch
+        // apart. key >= T  <=>  score > score(T), or score == score(T) and s <= index(T).
+        float tf[QPW], sqr[QPW];
+        uint32_t tix[QPW];
+#pragma unroll
+        for (int qi = 0; qi < QPW; ++qi) {
+          const uint64_t T = sm.thr[qbase + qi];
+          tf[qi] = key_score(T);  // -inf for T = 0: every key is taken
+          tix[qi] = T ? static_cast<uint32_t>(key_index(T)) : 0xFFFFFFFFu;
+          sqr[qi] = sm.sq[qbase + qi];
+        }
+        uint64_t* const dst0 = p.cand + static_cast<size_t>(row_base) * pitch + wl * p.seg_stride;
+        // Tiles whose keys all lie at or before the earlier query's position need no mask
+        // (every such key is also below Lk); only the diagonal tiles are masked. The sample pass
+        // reads every S-th key (map row v is key S v) and appends every valid one (T = 0).
+        const bool rows_ok = row_base + QPW - 1 < p.Lq;
+        const int n_plain = rows_ok ? min(nt, ((p.q_pos0 + row_base) / p.stride + 1) / C::BN) : 0;
+        auto lean_tile = [&](auto masked_tag) {
+          constexpr bool MASKED = decltype(masked_tag)::value;
+          const float sk = sk_next;
+          sk_next = __ldg(&p.k_scale[static_cast<size_t>(min(v + C::BN, p.nkeys - 1)) * p.stride]);
+          const int s = v * p.stride;  // the key's position
+          const bool got = mbar_wait(&sm.accfull[g], use & 1u, ctl, DETAIL_WAIT_ACCFULL);
+          good = good && got;
+          __syncwarp();
+          tc_fence_after();
+          float part[4][2];
+          lean_partials(taddr0, &sm.wq[qbase][0], lane & 3u, part);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.accempty[g]);
+          ++use;
+          float score_part[QPW];
+#pragma unroll
+          for (int qi = 0; qi < QPW; ++qi) {
+            const float col[4] = {part[0][qi], part[1][qi], part[2][qi], part[3][qi]};
+            score_part[qi] = slot_total(col, lane & 3u);
+          }
+#pragma unroll
+          for (int qi = 0; qi < QPW; ++qi) {
+            const float score = (score_part[qi] * sqr[qi]) * sk;
+            bool take = score > tf[qi] || (score == tf[qi] && static_cast<uint32_t>(s) <= tix[qi]);
+            if constexpr (MASKED) take = take && (row_base + qi < p.Lq) && (s <= p.q_pos0 + row_base + qi);
+            const uint32_t m = __ballot_sync(0xFFFFFFFFu, take);
+            if (m) {  // warp-uniform: most warps of a long row append nothing
+              const uint32_t pos = cw[qi] + __popc(m & lt);
+              if (take && pos < segcap) dst0[qi * pitch + pos] = make_key(score, static_cast<uint32_t>(s));
+              cw[qi] += __popc(m);
+            }
+          }
+          v += C::BN;
+        };
+        int tile = 0;
+        for (; tile < n_plain; ++tile) lean_tile(std::integral_constant<bool, false>{});
+        for (; tile < nt; ++tile) lean_tile(std::integral_constant<bool, true>{});
+      } else {
       for (int tile = 0; tile < nt; ++tile, v += C::BN) {
         const float sk = sk_next;
         sk_next = scale_of(v + C::BN);
@@ -368,65 +564,8 @@ __global__ void __launch_bounds__(PRoles<H, MODE>::THREADS, 1)
         good = good && got;
         __syncwarp();
         tc_fence_after();
-        // This warp's QPW * H columns in chunks of 32.
-        constexpr int NCH = QPW * H / 32;
         float score_part[QPW];
-        uint32_t ra[32], rb[32];
-        tmem_ld_32x32b_x32(taddr0, ra);
-        tmem_wait_ld_regs(ra);
-        if constexpr (H == 64) {
-          // 64 heads per query: packed FMA over head pairs, four float2 partial sums per query.
-          float2 acc[QPW][4];
-#pragma unroll
-          for (int qi = 0; qi < QPW; ++qi)
-#pragma unroll
-            for (int a = 0; a < 4; ++a) acc[qi][a] = make_float2(0.0f, 0.0f);
-#pragma unroll
-          for (int c = 0; c < NCH; ++c) {
-            uint32_t(&cur)[32] = (c & 1) ? rb : ra;
-            uint32_t(&nxt)[32] = (c & 1) ? ra : rb;
-            if (c + 1 < NCH) tmem_ld_32x32b_x32(taddr0 + (c + 1) * 32, nxt);
-            const int qi = c >> 1;
-#pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-              const int h = (c & 1) * 32 + j;
-              const float4 wv = *reinterpret_cast<const float4*>(&sm.wq[qbase + qi][h]);
-              const float r0 = __saturatef(__uint_as_float(cur[j + 0]) * 0x1p-25f);
-              const float r1 = __saturatef(__uint_as_float(cur[j + 1]) * 0x1p-25f);
-              const float r2 = __saturatef(__uint_as_float(cur[j + 2]) * 0x1p-25f);
-              const float r3 = __saturatef(__uint_as_float(cur[j + 3]) * 0x1p-25f);
-              const int a = QPW >= 4 ? ((j >> 2) & 1) * 2 : 0;  // fewer chains when registers are scarce
-              acc[qi][a] = __ffma2_rn(make_float2(wv.x, wv.y), make_float2(r0, r1), acc[qi][a]);
-              acc[qi][a + 1] = __ffma2_rn(make_float2(wv.z, wv.w), make_float2(r2, r3), acc[qi][a + 1]);
-            }
-            if (c + 1 < NCH) tmem_wait_ld_regs(nxt);
-          }
-#pragma unroll
-          for (int qi = 0; qi < QPW; ++qi)
-            score_part[qi] = ((acc[qi][0].x + acc[qi][0].y) + (acc[qi][1].x + acc[qi][1].y)) +
-                             ((acc[qi][2].x + acc[qi][2].y) + (acc[qi][3].x + acc[qi][3].y));
-        } else {
-          // 8 heads per query: one scalar chain per query, four queries per chunk.
-#pragma unroll
-          for (int qi = 0; qi < QPW; ++qi) score_part[qi] = 0.0f;
-#pragma unroll
-          for (int c = 0; c < NCH; ++c) {
-            uint32_t(&cur)[32] = (c & 1) ? rb : ra;
-            uint32_t(&nxt)[32] = (c & 1) ? ra : rb;
-            if (c + 1 < NCH) tmem_ld_32x32b_x32(taddr0 + (c + 1) * 32, nxt);
-#pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-              const int col = c * 32 + j;
-              const int qi = col / H, h = col % H;
-              const float4 wv = *reinterpret_cast<const float4*>(&sm.wq[qbase + qi][h]);
-              score_part[qi] = fmaf(wv.x, __saturatef(__uint_as_float(cur[j + 0]) * 0x1p-25f), score_part[qi]);
-              score_part[qi] = fmaf(wv.y, __saturatef(__uint_as_float(cur[j + 1]) * 0x1p-25f), score_part[qi]);
-              score_part[qi] = fmaf(wv.z, __saturatef(__uint_as_float(cur[j + 2]) * 0x1p-25f), score_part[qi]);
-              score_part[qi] = fmaf(wv.w, __saturatef(__uint_as_float(cur[j + 3]) * 0x1p-25f), score_part[qi]);
-            }
-            if (c + 1 < NCH) tmem_wait_ld_regs(nxt);
-          }
-        }
+        head_sums<H, QPW>(taddr0, &sm.wq[qbase], score_part);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.accempty[g]);
@@ -469,6 +608,7 @@ __global__ void __launch_bounds__(PRoles<H, MODE>::THREADS, 1)
             for (int qi = 0; qi < QPW; ++qi) cw[qi] = sm.wcnt[qbase + qi][wl];
           }
         }
+      }
       }
       ok = named_bar_and(1u + sub, 128, ok && good);
       if (!ok) break;
