@@ -192,20 +192,27 @@ dsa_status launch_prefill_finish(const uint64_t* cand, const uint32_t* counts,
 // the k-th largest key is a 6.5-sigma event, and otherwise at least k keys of the row are >= T.
 // A row with r >= n_s (short rows, n <= k) gets T = 0: every key is kept. (The lean pass checks
 // the count it actually appended and hands the rare failure to the exact pass.)
-// One warp per row: a radix select on the 64-bit keys with digits of up to 8 bits, starting at
-// the highest bit where the row's smallest and largest sampled key differ, with a warp-private
-// 256-bin histogram; no block-wide barrier.
+// Per prefill row (one warp), the lean pass's threshold: the sampled key of rank r (largest
+// first), by radix passes with 8-bit digits below the bits every sample shares. STAGED: the
+// row's samples are read from global memory once into the warp's shared-memory stage and the
+// passes read the stage (rows of up to kThrStageMax samples, eight warps per block); otherwise
+// every pass reads global memory with eight loads in flight per lane, which keeps many more
+// rows in flight than a stage of a long row's samples would allow.
 constexpr int kThrWarps = 8;
+constexpr uint32_t kThrStageMax = 1024;
 
+template <bool STAGED>
 __global__ void __launch_bounds__(32 * kThrWarps)
     prefill_sample_threshold_kernel(const uint64_t* __restrict__ cand, const uint32_t* __restrict__ counts,
                                     uint64_t* __restrict__ thr, uint32_t seg_stride, int rows, int q_pos0,
                                     int Lk, int topk) {
   __shared__ uint32_t hist_all[kThrWarps][256];
+  extern __shared__ uint64_t stage_all[];  // STAGED: kThrWarps x kThrStageMax keys
   const uint32_t lane = threadIdx.x & 31u, wi = threadIdx.x >> 5;
   const int row = blockIdx.x * kThrWarps + static_cast<int>(wi);
   if (row >= rows) return;  // warp-uniform; the block has no barrier
   uint32_t* hist = hist_all[wi];
+  uint64_t* stage = stage_all + (STAGED ? wi * kThrStageMax : 0u);
   const uint64_t* buf = cand + static_cast<size_t>(row) * 4u * seg_stride;
   uint32_t c[4];
 #pragma unroll
@@ -213,7 +220,8 @@ __global__ void __launch_bounds__(32 * kThrWarps)
     const uint32_t v = __ldcg(counts + static_cast<size_t>(row) * 4 + w);
     c[w] = v < seg_stride ? v : seg_stride;
   }
-  const uint32_t o1 = c[0], o2 = o1 + c[1], o3 = o2 + c[2], ns = o3 + c[3];
+  const uint32_t o1 = c[0], o2 = o1 + c[1], o3 = o2 + c[2];
+  const uint32_t ns = STAGED ? min(o3 + c[3], kThrStageMax) : o3 + c[3];
   const int keys = min(q_pos0 + row + 1, Lk);
   const double rho = static_cast<double>(topk) * ns / keys;
   const double rr = rho + 6.5 * sqrt(rho) + 1.0;
@@ -222,13 +230,12 @@ __global__ void __launch_bounds__(32 * kThrWarps)
     return;
   }
   const uint32_t r = static_cast<uint32_t>(ceil(rr));
-  auto key_at = [&](uint32_t e) {
+  auto global_at = [&](uint32_t e) {
     const uint32_t w = (e >= o1 ? 1u : 0u) + (e >= o2 ? 1u : 0u) + (e >= o3 ? 1u : 0u);
     const uint32_t start = e >= o3 ? o3 : (e >= o2 ? o2 : (e >= o1 ? o1 : 0u));
     return __ldcg(buf + w * seg_stride + (e - start));
   };
-  // Bits common to every sampled key are fixed from the start.
-  // Eight independent loads in flight per lane in every pass over the samples.
+  // First pass: the samples' range (and, STAGED, the stage).
   constexpr int kBatch = 8;
   uint64_t mn = ~0ull, mx = 0ull;
   for (uint32_t e0 = 0; e0 < ns; e0 += 32 * kBatch) {
@@ -236,12 +243,13 @@ __global__ void __launch_bounds__(32 * kThrWarps)
 #pragma unroll
     for (int i = 0; i < kBatch; ++i) {
       const uint32_t e = e0 + i * 32 + lane;
-      v[i] = e < ns ? key_at(e) : 0ull;
+      v[i] = e < ns ? global_at(e) : 0ull;
     }
 #pragma unroll
     for (int i = 0; i < kBatch; ++i) {
       const uint32_t e = e0 + i * 32 + lane;
       if (e < ns) {
+        if (STAGED) stage[e] = v[i];
         mn = v[i] < mn ? v[i] : mn;
         mx = v[i] > mx ? v[i] : mx;
       }
@@ -253,6 +261,8 @@ __global__ void __launch_bounds__(32 * kThrWarps)
     mn = a < mn ? a : mn;
     mx = b > mx ? b : mx;
   }
+  __syncwarp();
+  // Bits common to every sampled key are fixed from the start.
   int hb = 63 - __clzll(static_cast<long long>(mn ^ mx));
   uint64_t mask = (hb >= 63) ? 0ull : ~((2ull << hb) - 1ull);
   uint64_t prefix = mx & mask;
@@ -263,18 +273,25 @@ __global__ void __launch_bounds__(32 * kThrWarps)
 #pragma unroll
     for (int i = 0; i < 8; ++i) hist[lane * 8 + i] = 0u;
     __syncwarp();
-    for (uint32_t e0 = 0; e0 < ns; e0 += 32 * kBatch) {
-      uint64_t v[kBatch];
-#pragma unroll
-      for (int i = 0; i < kBatch; ++i) {
-        const uint32_t e = e0 + i * 32 + lane;
-        v[i] = e < ns ? key_at(e) : 0ull;
+    if constexpr (STAGED) {
+      for (uint32_t e = lane; e < ns; e += 32) {
+        const uint64_t v = stage[e];
+        if ((v & mask) == prefix) atomicAdd(&hist[static_cast<uint32_t>(v >> shift) & dmask], 1u);
       }
+    } else {
+      for (uint32_t e0 = 0; e0 < ns; e0 += 32 * kBatch) {
+        uint64_t v[kBatch];
 #pragma unroll
-      for (int i = 0; i < kBatch; ++i) {
-        const uint32_t e = e0 + i * 32 + lane;
-        if (e < ns && (v[i] & mask) == prefix)
-          atomicAdd(&hist[static_cast<uint32_t>(v[i] >> shift) & dmask], 1u);
+        for (int i = 0; i < kBatch; ++i) {
+          const uint32_t e = e0 + i * 32 + lane;
+          v[i] = e < ns ? global_at(e) : 0ull;
+        }
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i) {
+          const uint32_t e = e0 + i * 32 + lane;
+          if (e < ns && (v[i] & mask) == prefix)
+            atomicAdd(&hist[static_cast<uint32_t>(v[i] >> shift) & dmask], 1u);
+        }
       }
     }
     __syncwarp();
@@ -322,10 +339,19 @@ dsa_status launch_prefill_sample_threshold(const uint64_t* cand, const uint32_t*
                                            uint64_t* thr, uint32_t seg_stride, int rows,
                                            int q_pos0, int Lk, int topk, uint32_t max_samples,
                                            cudaStream_t stream) {
-  (void)max_samples;
+  // A row holds at most max_samples sampled keys (and at most its four segments).
+  const uint32_t most = max_samples < 4u * seg_stride ? max_samples : 4u * seg_stride;
   const int grid = (rows + kThrWarps - 1) / kThrWarps;
-  prefill_sample_threshold_kernel<<<grid, 32 * kThrWarps, 0, stream>>>(cand, counts, thr, seg_stride, rows,
-                                                                      q_pos0, Lk, topk);
+  if (most <= kThrStageMax) {
+    constexpr size_t smem = static_cast<size_t>(kThrWarps) * kThrStageMax * sizeof(uint64_t);
+    if (cudaFuncSetAttribute(prefill_sample_threshold_kernel<true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    prefill_sample_threshold_kernel<true><<<grid, 32 * kThrWarps, smem, stream>>>(cand, counts, thr, seg_stride,
+                                                                                rows, q_pos0, Lk, topk);
+  } else
+    prefill_sample_threshold_kernel<false><<<grid, 32 * kThrWarps, 0, stream>>>(cand, counts, thr, seg_stride,
+                                                                              rows, q_pos0, Lk, topk);
   return cuda_status(cudaGetLastError());
 }
 
