@@ -1,12 +1,15 @@
 // Cross-layer top-k overlap: C[i][j] = sum over rows of |T_i(row) ∩ T_j(row)|.
 //
-// Integer work bound by reading the N index tensors (N * rows * topk * 4 bytes, each byte once).
-// A CTA walks rows. For a row it marks every layer's indices in per-layer shared-memory bitmaps
-// over the row's index range (all of a row's loads in flight before the first mark), counts
-// each pair (i <= j) as the popcount of the AND of the two bitmaps, and clears the bitmaps. When the N bitmaps over [0, n_keys) do not fit in shared
-// memory, one bitmap at a time is built and the other layers' entries are probed against it.
-// Counts accumulate in shared 64-bit counters per CTA and are added to the output once per CTA;
-// a finishing kernel mirrors the upper triangle and forms C / V.
+// Integer work bound by reading the N index tensors (N * rows * topk * 4 bytes, each byte once)
+// and by the shared-memory marks: every listed index sets one bit with a shared atomic, about
+// 3.5 bank wavefronts per warp instruction for random indices. Small CTAs (four warps, up to
+// eight per SM) walk rows independently, so while some mark, others load or count. For a row a
+// CTA marks every layer's indices in per-layer shared-memory bitmaps over the row's index range,
+// one layer's loads in flight at a time, counts each pair (i <= j) as the popcount of the AND of
+// the two bitmaps and clears the bitmaps. When the N bitmaps over [0, n_keys) do not fit in
+// shared memory, one bitmap at a time is built and the other layers' entries are probed against
+// it. Counts accumulate in shared 64-bit counters per CTA and are added to the output once per
+// CTA; a finishing kernel mirrors the upper triangle and forms C / V.
 #include "common.cuh"
 #include "internal.h"
 
@@ -20,26 +23,26 @@ struct OverlapParams {
   WsHeader* hdr;
 };
 
-constexpr int kOverlapThreads = 256;
+constexpr int kOverlapThreads = 128;
+constexpr int kOverlapMinBlocks = 8;  // CTAs per SM the register budget is sized for
 constexpr size_t kOverlapSmemBudget = 200 * 1024;
 
 __device__ __forceinline__ unsigned long long* overlap_acc(uint8_t* smem) {
   return reinterpret_cast<unsigned long long*>(smem);
 }
 
-// All N bitmaps resident: bits[i][w], W words per layer. A row's indices are loaded for up to
-// kOvGroup layers at once (every load in flight before the first bitmap update), then marked.
-// With N <= kOvGroup (SMALL) each thread keeps its pair counts in registers across rows and
-// reduces them once at the end (and every kOvFlushRows rows, so a 32-bit count cannot wrap);
-// otherwise each row's pair counts are reduced per warp into the shared counters.
+// All N bitmaps resident: bits[i][w], W words per layer. With N <= kOvGroup (SMALL) each
+// thread keeps its pair counts in registers across rows, two 16-bit counts per register, and
+// reduces them into the shared counters before a count can wrap (a row adds at most 32 per
+// word a thread counts) and at the end; otherwise each row's pair counts are reduced per warp
+// into the shared counters. VEC: rows start 16-byte aligned, indices are loaded as int4.
 constexpr int kOvGroup = 8;
 constexpr int kOvPerThread = DSA_MAX_TOPK / kOverlapThreads;  // indices per thread per layer
 constexpr int kOvPairs = kOvGroup * (kOvGroup + 1) / 2;
-constexpr int kOvFlushRows = 1 << 16;
-static_assert(DSA_MAX_TOPK % kOverlapThreads == 0, "indices per thread");
+static_assert(DSA_MAX_TOPK % (4 * kOverlapThreads) == 0, "indices per thread");
 
-template <bool SMALL>
-__global__ void __launch_bounds__(kOverlapThreads)
+template <bool SMALL, bool VEC>
+__global__ void __launch_bounds__(kOverlapThreads, kOverlapMinBlocks)
     overlap_bitmaps_kernel(const __grid_constant__ OverlapParams p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const int N = p.N;
@@ -54,56 +57,63 @@ __global__ void __launch_bounds__(kOverlapThreads)
   if (threadIdx.x == 0) *row_max = -1;
   __syncthreads();
   const uint32_t lane = threadIdx.x & 31u;
-  uint32_t creg[kOvPairs];
+  // Pair q's count in half q & 1 of creg[q / 2].
+  uint32_t creg[(kOvPairs + 1) / 2];
 #pragma unroll
-  for (int q = 0; q < kOvPairs; ++q) creg[q] = 0u;
+  for (int q = 0; q < (kOvPairs + 1) / 2; ++q) creg[q] = 0u;
+  const int words_pt = (W + kOverlapThreads - 1) / kOverlapThreads;
+  const int flush_rows = 65535 / (32 * words_pt);  // >= 1: W <= 51200 words in the budget
   // Adds the register pair counts into the shared counters (all threads of the CTA).
   auto flush_creg = [&]() {
 #pragma unroll
     for (int q = 0; q < kOvPairs; ++q) {
-      uint32_t c = creg[q];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xFFFFFFFFu, c, o);
+      const uint32_t c = __reduce_add_sync(0xFFFFFFFFu, (creg[q >> 1] >> (16 * (q & 1))) & 0xFFFFu);
       if (lane == 0 && c) atomicAdd(&acc[q], static_cast<unsigned long long>(c));
-      creg[q] = 0u;
     }
+#pragma unroll
+    for (int q = 0; q < (kOvPairs + 1) / 2; ++q) creg[q] = 0u;
   };
   int it = 0;
   for (int row = blockIdx.x; row < p.rows; row += gridDim.x) {
     const size_t off = static_cast<size_t>(row) * p.topk;
     int local_max = -1;
     uint32_t valid0 = 0;
-    for (int i0 = 0; i0 < N; i0 += kOvGroup) {
-      int32_t v[kOvGroup][kOvPerThread];
+    for (int i = 0; i < N; ++i) {
+      int32_t v[kOvPerThread];
+      if constexpr (VEC) {
+        const int4* src = reinterpret_cast<const int4*>(p.layers[i] + off);
 #pragma unroll
-      for (int ii = 0; ii < kOvGroup; ++ii) {
-        const int i = i0 + ii;
+        for (int q4 = 0; q4 < kOvPerThread / 4; ++q4) {
+          const int e4 = static_cast<int>(threadIdx.x) + q4 * kOverlapThreads;
+          const int4 t = 4 * e4 < p.topk ? __ldcs(src + e4) : make_int4(-1, -1, -1, -1);
+          v[4 * q4 + 0] = t.x;
+          v[4 * q4 + 1] = t.y;
+          v[4 * q4 + 2] = t.z;
+          v[4 * q4 + 3] = t.w;
+        }
+      } else {
 #pragma unroll
         for (int q = 0; q < kOvPerThread; ++q) {
           const int e = static_cast<int>(threadIdx.x) + q * kOverlapThreads;
-          v[ii][q] = (i < N && e < p.topk) ? __ldcs(p.layers[i] + off + e) : -1;
+          v[q] = e < p.topk ? __ldcs(p.layers[i] + off + e) : -1;
         }
       }
+      uint32_t* bi = bits + i * W;
 #pragma unroll
-      for (int ii = 0; ii < kOvGroup; ++ii) {
-        uint32_t* bi = bits + (i0 + ii) * W;
-#pragma unroll
-        for (int q = 0; q < kOvPerThread; ++q) {
-          const int32_t x = v[ii][q];
-          if (x >= 0 && x < p.n_keys) {
-            atomicOr(&bi[x >> 5], 1u << (x & 31));
-            local_max = x > local_max ? x : local_max;
-            if (i0 + ii == 0) ++valid0;
-          } else if (x != -1) {
-            record_error(p.hdr, DSA_ERR_DEVICE, DETAIL_BAD_INDEX);
-          }
+      for (int q = 0; q < kOvPerThread; ++q) {
+        const int32_t x = v[q];
+        if (x >= 0 && x < p.n_keys) {
+          atomicOr(&bi[x >> 5], 1u << (x & 31));
+          local_max = x > local_max ? x : local_max;
+          if (i == 0) ++valid0;
+        } else if (x != -1) {
+          record_error(p.hdr, DSA_ERR_DEVICE, DETAIL_BAD_INDEX);
         }
       }
     }
     local_max = __reduce_max_sync(0xFFFFFFFFu, local_max);  // one shared atomic per warp
     if (lane == 0 && local_max >= 0) atomicMax(row_max, local_max);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) valid0 += __shfl_xor_sync(0xFFFFFFFFu, valid0, o);
+    valid0 = __reduce_add_sync(0xFFFFFFFFu, valid0);
     if (lane == 0 && valid0) atomicAdd(&acc[npairs], static_cast<unsigned long long>(valid0));
     __syncthreads();
     const int wr = (*row_max >> 5) + 1;  // words that can hold a mark in this row
@@ -116,7 +126,8 @@ __global__ void __launch_bounds__(kOverlapThreads)
 #pragma unroll
         for (int i = 0; i < kOvGroup; ++i)
 #pragma unroll
-          for (int j = i; j < kOvGroup; ++j, ++q) creg[q] += __popc(m[i] & m[j]);
+          for (int j = i; j < kOvGroup; ++j, ++q)
+            creg[q >> 1] += static_cast<uint32_t>(__popc(m[i] & m[j])) << (16 * (q & 1));
       }
     } else {
       int pair = 0;
@@ -126,8 +137,7 @@ __global__ void __launch_bounds__(kOverlapThreads)
           const uint32_t* bj = bits + j * W;
           uint32_t c = 0;
           for (int w = threadIdx.x; w < wr; w += kOverlapThreads) c += __popc(bi[w] & bj[w]);
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xFFFFFFFFu, c, o);
+          c = __reduce_add_sync(0xFFFFFFFFu, c);
           if (lane == 0 && c) atomicAdd(&acc[pair], static_cast<unsigned long long>(c));
         }
       }
@@ -137,7 +147,7 @@ __global__ void __launch_bounds__(kOverlapThreads)
       for (int w = threadIdx.x; w < wr; w += kOverlapThreads) bits[i * W + w] = 0u;
     if (threadIdx.x == 0) *row_max = -1;
     if constexpr (SMALL) {
-      if (++it == kOvFlushRows) {
+      if (++it == flush_rows) {
         flush_creg();
         it = 0;
       }
@@ -267,10 +277,14 @@ dsa_status launch_overlap(const int32_t* const* layer_idx, int32_t n_layers, int
                                                : static_cast<size_t>(n_layers) * (n_layers + 1) / 2;
     const size_t smem_all = (npairs + 1) * 8 + 16 + static_cast<size_t>(n_layers) * words * 4;
     dsa_status st;
-    if (smem_all <= kOverlapSmemBudget && n_layers <= kOvGroup)
-      st = launch_overlap_kernel(overlap_bitmaps_kernel<true>, p, smem_all, rows, stream, num_sms);
-    else if (smem_all <= kOverlapSmemBudget)
-      st = launch_overlap_kernel(overlap_bitmaps_kernel<false>, p, smem_all, rows, stream, num_sms);
+    bool vec = topk % 4 == 0;
+    for (int i = 0; i < n_layers; ++i) vec = vec && (reinterpret_cast<uintptr_t>(layer_idx[i]) & 15u) == 0;
+    const bool small = n_layers <= kOvGroup;
+    if (smem_all <= kOverlapSmemBudget)
+      st = small ? (vec ? launch_overlap_kernel(overlap_bitmaps_kernel<true, true>, p, smem_all, rows, stream, num_sms)
+                        : launch_overlap_kernel(overlap_bitmaps_kernel<true, false>, p, smem_all, rows, stream, num_sms))
+                 : (vec ? launch_overlap_kernel(overlap_bitmaps_kernel<false, true>, p, smem_all, rows, stream, num_sms)
+                        : launch_overlap_kernel(overlap_bitmaps_kernel<false, false>, p, smem_all, rows, stream, num_sms));
     else
       st = launch_overlap_kernel(overlap_probe_kernel, p, (nn + 1) * 8 + words * 4, rows, stream,
                                  num_sms);

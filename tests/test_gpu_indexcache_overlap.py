@@ -102,7 +102,8 @@ def _random_rows(R, topk, n_keys, N, seed, base=None):
 
 
 @pytest.mark.parametrize("N,R,topk,n_keys", [(4, 300, 64, 300), (8, 100, 2048, 5000), (3, 1, 5, 5),
-                                                (12, 60, 256, 2000), (5, 200, 130, 1000)])
+                                                (12, 60, 256, 2000), (5, 200, 130, 1000),
+                                                (9, 40, 130, 700), (8, 3000, 16, 64)])
 def test_overlap_counts_bit_exact(N, R, topk, n_keys):
     layers = _random_rows(R, topk, n_keys, N, seed=N * R)
     counts, valid, overlap = B.topk_overlap([torch.from_numpy(T).cuda() for T in layers], n_keys)
@@ -149,6 +150,50 @@ def test_overlap_wide_index_range_uses_probe_path():
         layers.append(np.where(drop, -1, first).astype(np.int32))
     layers.append(np.concatenate([first[:, : topk // 2], np.full((R, topk - topk // 2), -1, np.int32)], 1))
     counts, valid, overlap = B.topk_overlap([torch.from_numpy(T).cuda() for T in layers], n_keys)
+    torch.cuda.synchronize()
+    ref_c, ref_v, ref_o = O.topk_overlap(layers)
+    assert counts.cpu().numpy().astype(np.uint64).tolist() == ref_c.tolist()
+    assert int(valid.item()) == ref_v
+
+
+def test_overlap_register_counts_flush_between_rows():
+    """n_keys = 300000 sizes the bitmaps (and so the words a thread may count per row) for a wide
+    range while every index stays below 3000: the 16-bit register pair counts are then flushed
+    into the shared counters every few rows, and 6000 rows give every CTA several flushes."""
+    N, R, topk, n_keys, span = 4, 6000, 64, 300000, 3000
+    rng = np.random.default_rng(23)
+    base = np.stack([rng.choice(span, size=topk, replace=False) for _ in range(R)]).astype(np.int32)
+    layers = [base]
+    for i in range(1, N):
+        other = np.stack([rng.choice(span, size=topk, replace=False) for _ in range(R)]).astype(np.int32)
+        keep = rng.random(base.shape) < 0.6
+        mixed = np.where(keep, base, -2)
+        rows = []
+        for t in range(R):   # layer i: ~60% of layer 0's row, topped up with distinct other keys
+            kept = mixed[t][mixed[t] >= 0]
+            extra = [x for x in other[t] if x not in set(kept)][: topk - len(kept)]
+            rows.append(np.concatenate([kept, np.array(extra, dtype=np.int32)]))
+        layers.append(np.stack(rows).astype(np.int32))
+    counts, valid, overlap = B.topk_overlap([torch.from_numpy(T).cuda() for T in layers], n_keys)
+    torch.cuda.synchronize()
+    ref_c, ref_v, ref_o = O.topk_overlap(layers)
+    assert counts.cpu().numpy().astype(np.uint64).tolist() == ref_c.tolist()
+    assert int(valid.item()) == ref_v
+    assert np.array_equal(overlap.cpu().numpy(), ref_o)
+
+
+def test_overlap_unaligned_rows_use_scalar_loads():
+    """Rows of layers that start off a 16-byte boundary (a view one element into a buffer) are
+    read with scalar loads; counts match the oracle."""
+    N, R, topk, n_keys = 3, 200, 64, 500
+    layers = _random_rows(R, topk, n_keys, N, seed=31)
+    views = []
+    for T in layers:
+        buf = torch.full((R * topk + 1,), -1, dtype=torch.int32, device="cuda")
+        buf[1:] = torch.from_numpy(T).cuda().reshape(-1)
+        views.append(buf[1:].view(R, topk))
+    assert views[0].data_ptr() % 16 != 0
+    counts, valid, overlap = B.topk_overlap(views, n_keys)
     torch.cuda.synchronize()
     ref_c, ref_v, ref_o = O.topk_overlap(layers)
     assert counts.cpu().numpy().astype(np.uint64).tolist() == ref_c.tolist()
