@@ -311,34 +311,85 @@ def run_long(args, world, rank, device, peaks, peak_kind):
 
 def run_long_e2e(args, world, lp, pattern, stream):
     """The headline step end to end through the public API: every step copies the F layers'
-    inputs from pinned host memory to the device and every F layer's index rows back."""
+    inputs from pinned host memory to the device and every F layer's index rows back.
+
+    The copies are pipelined with the chunk-major compute, as a serving loop would: chunk c+1's
+    query rows and new key rows go up on a copy stream while chunk c is scored (they are rows
+    chunk c does not read), and each F layer's index rows of chunk c go down on a second copy
+    stream as soon as that layer has run, from one of two alternating sets of per-layer chunk
+    buffers (a set is rewritten only after its previous copies have landed). The step ends when
+    its last rows are on the host."""
     f_layers = [l for l, c in enumerate(pattern) if c == "F"]
+    f_index = {l: j for j, l in enumerate(f_layers)}
     names = ("q", "q_scale", "w", "k", "k_scale")
     host_in = {l: {n: getattr(lp.layers[l], n).cpu().pin_memory() for n in names} for l in f_layers}
     host_out = {l: torch.empty(lp.L, lp.topk, dtype=torch.int32).pin_memory() for l in f_layers}
     h2d = sum(t.numel() * t.element_size() for d in host_in.values() for t in d.values())
     d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    n_chunks, n_full = len(lp.chunks), len(f_layers)
+    bufs = [[torch.empty(lp.chunk, lp.topk, dtype=torch.int32, device=lp.device) for _ in range(n_full)]
+            for _ in range(2)]
+    up, down = torch.cuda.Stream(lp.device), torch.cuda.Stream(lp.device)
+    ev_up = [torch.cuda.Event() for _ in range(n_chunks)]
+    ev_run = [[torch.cuda.Event() for _ in range(n_full)] for _ in range(n_chunks)]
+    ev_down = [[torch.cuda.Event() for _ in range(n_full)] for _ in range(2)]
+    used = [False, False]
 
-    def after(ci, l):
-        if pattern[l] == "F":
-            c0, c1 = lp.chunks[ci]
-            host_out[l][c0:c1].copy_(lp.out[: c1 - c0], non_blocking=True)
+    def upload(ci):
+        c0, c1 = lp.chunks[ci]
+        with torch.cuda.stream(up):
+            for l in f_layers:
+                dev, host = lp.layers[l], host_in[l]
+                for n in names:
+                    getattr(dev, n)[c0:c1].copy_(host[n][c0:c1], non_blocking=True)
+        ev_up[ci].record(up)
 
     def e2e_step():
-        for l in f_layers:
-            for n in names:
-                getattr(lp.layers[l], n).copy_(host_in[l][n], non_blocking=True)
-        lp.step(pattern, after_chunk_layer=after)
+        up.wait_stream(stream)  # the previous step's compute still reads these inputs
+        used[0] = used[1] = False
+        upload(0)
+        for ci, (c0, c1) in enumerate(lp.chunks):
+            if ci + 1 < n_chunks:
+                upload(ci + 1)
+            stream.wait_event(ev_up[ci])
+            par = ci % 2
+            if used[par]:
+                for e in ev_down[par]:
+                    stream.wait_event(e)
+            used[par] = True
+            fb = [b[: c1 - c0] for b in bufs[par]]
+
+            def after(l, ptr, ci=ci, c0=c0, c1=c1, par=par, fb=fb):
+                if pattern[l] != "F":
+                    return
+                j = f_index[l]
+                ev_run[ci][j].record(stream)
+                down.wait_event(ev_run[ci][j])
+                with torch.cuda.stream(down):
+                    host_out[l][c0:c1].copy_(fb[j], non_blocking=True)
+                ev_down[par][j].record(down)
+
+            views = [v if pattern[l] == "F" else None for l, v in enumerate(lp.views[ci])]
+            lp.B.indexcache_run(pattern, views, lp.topk, f_bufs=fb, keep_all=True, q_pos0=c0,
+                                workspace=lp.ws, after_layer=after)
+        stream.wait_stream(down)
 
     e2e_step()
     torch.cuda.synchronize()
     barrier(world, lp.device)
     ms = max_over_ranks(timed(stream, e2e_step, args.e2e_steps), world, lp.device)
     pairs = sum_over_ranks(lp.pairs(pattern) * args.e2e_steps, world, lp.device)
-    del host_in, host_out
+    # the indices that came back are the device's: spot-check the last chunk of every F layer
+    c0, c1 = lp.chunks[-1]
+    par = (n_chunks - 1) % 2
+    for l in f_layers:
+        if not torch.equal(host_out[l][c0:c1], bufs[par][f_index[l]][: c1 - c0].cpu()):
+            raise RuntimeError(f"e2e: host copy of layer {l} differs from the device buffer")
+    del host_in, host_out, bufs
     return {"value": pairs / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "steps": args.e2e_steps,
-            "ms_per_step": ms / args.e2e_steps}
+            "ms_per_step": ms / args.e2e_steps,
+            "copies": "pipelined with the compute on two copy streams (pinned host buffers)"}
 
 
 # DRAM bytes (read + write) of the lean pass (prefill_indexer_kernel<64, 128, 1>, the dominant

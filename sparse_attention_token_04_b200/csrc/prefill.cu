@@ -12,11 +12,14 @@
 //               128-column accumulators in the sample and lean modes and two 256-column ones in
 //               the exact mode, so the epilogue of one overlaps the MMAs of the others;
 //   warps 4..   four epilogue warps per accumulator (16 in the sample and lean modes, 8 in the
-//               exact mode), one per TMEM lane quarter. Thread = key (its TMEM lane): it reads
-//               the key's H head dot products of each query, applies ReLU, the head weights,
-//               then the query and key scales, masks s > t, and appends the keys it keeps to
-//               its warp's segment of the query's buffer (no atomics: the segment's count
-//               lives in a register of the warp).
+//               exact mode), one per TMEM lane quarter. In the exact mode a thread owns one
+//               key (its TMEM lane) and reads all H head dot products of each query; in the
+//               sample and lean modes (H = 64) a thread reads 16 lanes x 256 bits at a time,
+//               i.e. a quarter of the heads of four keys, and a four-thread reduce-scatter
+//               leaves it the full head sum of one key. The epilogue applies ReLU, the head
+//               weights, then the query and key scales, masks s > t, and appends the keys it
+//               keeps to its warp's segment of the query's buffer (no atomics: the segment's
+//               count lives in a register of the warp).
 //
 // The same kernel runs in three modes:
 //   sample  every S-th key only (a strided tensor map), every valid key appended: a uniform
