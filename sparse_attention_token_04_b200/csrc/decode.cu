@@ -19,7 +19,9 @@
 //              request's global histogram when the segment ends. The next request's head
 //              weights and query scale are loaded a segment ahead.
 // decode_collect_kernel and decode_rank_kernel (topk.cu) then select and order each request's
-// top-k.
+// top-k. Before the scoring kernel, decode_clear_kernel zeroes the histograms and the collection
+// state; the scoring kernel is its programmatic dependent (its prologue and first tiles overlap
+// the clear) and waits for it before its first histogram add and before it exits.
 #include <algorithm>
 #include <atomic>
 
@@ -265,6 +267,7 @@ __global__ void __launch_bounds__(192)
       sq_next = __ldg(&p.q_scale[b]);
     }
     auto flush_hist = [&](int req) {
+      grid_dependency_wait();  // the histograms are zero (decode_clear_kernel has completed)
       uint32_t* gbins = p.bins + static_cast<size_t>(req) * kScoreBins;
       for (int i = rank; i < kScoreBins; i += 128) {
         const uint32_t c = sm.hist[i];
@@ -349,12 +352,22 @@ __global__ void __launch_bounds__(192)
     }
     if (j > 0) flush_hist(b - 1);
   }
+  // Every CTA waits for the clear before it exits, so the kernels after this one, which wait
+  // for this grid only, find the histograms and the collection state cleared.
+  grid_dependency_wait();
   __syncthreads();
   grid_launch_dependents();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 128);
   }
+}
+
+// Zeroes the per-request histograms and collection state (n words) and lets the scoring kernel
+// launch at once.
+__global__ void __launch_bounds__(256) decode_clear_kernel(uint32_t* __restrict__ words, uint32_t n) {
+  grid_launch_dependents();
+  for (uint32_t e = blockIdx.x * 256u + threadIdx.x; e < n; e += gridDim.x * 256u) words[e] = 0u;
 }
 
 // CTAs of the scoring kernel that fit on one SM at once (the persistent grid is this many per
@@ -414,13 +427,26 @@ static dsa_status launch_decode_t(const DecodeLaunch& a) {
   p.scores = reinterpret_cast<float*>(base + lay.scores);
   p.bins = reinterpret_cast<uint32_t*>(base + lay.bins);
   p.budget_ns = a.budget_ns;
-  // Histograms and collection state, cleared together.
-  if (cudaMemsetAsync(p.bins, 0, lay.cand - lay.bins, a.stream) != cudaSuccess) return DSA_ERR_CUDA;
+  // Histograms and collection state, cleared together by a small kernel whose programmatic
+  // dependent is the scoring kernel.
+  const uint32_t n_clear = static_cast<uint32_t>((lay.cand - lay.bins) / sizeof(uint32_t));
+  const uint32_t clear_grid = std::min<uint32_t>((n_clear + 1023u) / 1024u, 128u);
+  decode_clear_kernel<<<clear_grid, 256, 0, a.stream>>>(p.bins, n_clear);
+  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
   const int per_sm = decode_ctas_per_sm(reinterpret_cast<const void*>(kern), C::THREADS, smem);
   if (per_sm < 1) return DSA_ERR_CUDA;
   const int grid = per_sm * (a.num_sms > 0 ? a.num_sms : 1);
-  kern<<<grid, C::THREADS, smem, a.stream>>>(tq, tk, p);
-  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = a.stream;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, tq, tk, p) != cudaSuccess) return DSA_ERR_CUDA;
   return launch_decode_topk(a.ws, lay, max_len, a.seq_lens, a.B, a.topk, a.out_idx, a.out_score,
                             a.budget_ns, a.stream);
 }
