@@ -661,12 +661,15 @@ __global__ void __launch_bounds__(PRoles<H, MODE>::THREADS, 1)
   }
 }
 
-// Key stride S of the sample pass for top-k over rows of up to Lk keys: about k / S >= 128
+// Key stride S of the sample pass for top-k over rows of up to Lk keys: about k / S >= 64
 // sampled keys lie above a row's k-th largest key, and a row's sample (ceil(Lk / S) keys)
-// fits its buffer. 1 means no sample pass: every block runs in the exact mode.
+// fits its buffer. 1 means no sample pass: every block runs in the exact mode. The sample pass
+// and the threshold cost about Lk / S per row, while the keys a row keeps above its threshold
+// grow only as k + 6.5 sqrt(k S); long rows (Lk >= 24576) take twice the stride.
 static int sample_stride(int topk, int Lk, uint32_t seg_stride) {
-  const int S = topk / 128;
+  int S = topk / 128;
   if (S < 2) return 1;
+  if (Lk >= 24576) S *= 2;
   const int64_t room = 4 * static_cast<int64_t>(seg_stride) - 4 * 32;  // tiles end on 32-key boundaries
   const int min_s = static_cast<int>((static_cast<int64_t>(Lk) + room - 1) / room);
   return S > min_s ? S : min_s;
