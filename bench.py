@@ -51,6 +51,8 @@ FP8_PER_BF16 = 2.0  # nominal dense FP8 / BF16 tensor throughput ratio on B200
 # Kernel launches of one dsa_indexer_prefill call with top-k 2048: sample pass, per-row sample
 # threshold, lean pass, exact pass (exits at once when the lean pass marked no block), finish.
 PREFILL_LAUNCHES_PER_CALL = 5
+# decode: the histogram clear, the scoring kernel, the collection pass and the rank pass
+DECODE_LAUNCHES_PER_CALL = 4
 
 
 # ------------------------------------------------------------------------------------------
@@ -537,8 +539,8 @@ def run_decode(args, world, rank, device, peaks):
                         "searched 1/4 pattern (12 indexer layers)",
             "value": pairs / (ms / 1e3), "unit": UNIT, "ms_per_step": ms / args.decode_steps,
             "steps": args.decode_steps, "keys_per_layer": keys,
-            "roofline": {"kernel": "dsa_indexer_decode (decode_indexer_kernel + decode_collect_kernel "
-                                   "+ decode_rank_kernel)",
+            "roofline": {"kernel": "dsa_indexer_decode (decode_clear_kernel + decode_indexer_kernel + "
+                                   "decode_collect_kernel + decode_rank_kernel)",
                          "bound": "hbm", "achieved": gbs, "peak": float(peaks["hbm_gbs"]),
                          "unit": "GB/s", "frac": gbs / float(peaks["hbm_gbs"]),
                          "traffic": (None if DECODE_SCORING_DRAM_BYTES_PER_KEY is None
@@ -547,7 +549,7 @@ def run_decode(args, world, rank, device, peaks):
                          "algorithmic_per_launch": f"{bytes_per_launch} B (d+4 per key + per-request "
                                                    "q/w/scale/table/out)",
                          "launch_ms": launch_ms},
-            "gpu_launches": 3 * n_full * args.decode_steps}
+            "gpu_launches": DECODE_LAUNCHES_PER_CALL * n_full * args.decode_steps}
 
 
 def run_mli_decode(args, world, rank, device):
