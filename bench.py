@@ -396,12 +396,12 @@ def run_long_e2e(args, world, lp, pattern, stream):
 
 # DRAM bytes (read + write) of the lean pass (prefill_indexer_kernel<64, 128, 1>, the dominant
 # launch) over the 25 chunk calls of one 200000-token indexer layer, from one ncu capture of the
-# current kernel (dram__bytes_read.sum 2.134e9 + dram__bytes_write.sum 3.979e9): q read once
-# (1.64 GB), key tiles re-read per chunk, and the appended candidates written.
-PREFILL_LEAN_TRAFFIC_PER_LAYER = 2.134e9 + 3.979e9
+# current kernel and sample stride (dram__bytes_read.sum 2.139e9 + dram__bytes_write.sum
+# 4.517e9): q read once (1.64 GB), key tiles re-read per chunk, and the appended candidates written.
+PREFILL_LEAN_TRAFFIC_PER_LAYER = 2.139e9 + 4.517e9
 PREFILL_LEAN_TRAFFIC_SOURCE = ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum of the 25 lean-pass launches "
-                               "of one 200000-token layer (all 25 chunks, seed 5), summed; the whole call's other "
-                               "launches add 4.1e10 B, 2.5e10 of them the sample threshold's re-reads")
+                               "of one 200000-token layer (all 25 chunks, seed 5), summed; the call's other launches "
+                               "add 2.7e10 B, 1.4e10 of them the sample threshold's re-reads")
 
 
 # ------------------------------------------------------------------------------------------
