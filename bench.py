@@ -626,7 +626,7 @@ def run_mli_decode(args, world, rank, device):
 
 # DRAM bytes (read + write) per cached key of decode_indexer_kernel from one ncu capture of this
 # workload, or None when the kernel changed after the capture.
-DECODE_SCORING_DRAM_BYTES_PER_KEY = 5.034e8 / 3737801
+DECODE_SCORING_DRAM_BYTES_PER_KEY = 5.019e8 / 3737801
 DECODE_TRAFFIC_SOURCE = ("decode_indexer_kernel DRAM read+write per cached key from one ncu capture "
                          "of this workload (SpeedOfLight/MemoryWorkloadAnalysis sections), times the "
                          "keys of one launch")

@@ -264,6 +264,8 @@ DSA_API dsa_status indexcache_run_lagged(const char* pattern, int32_t n_layers,
  * out_valid  [1] u64: V = number of non-negative entries of layer 0.
  * out_overlap [n_layers][n_layers] f64 = C / V, or NULL.
  * An entry outside [-1, n_keys) is skipped and recorded as DSA_ERR_DEVICE.
+ * rows >= 0; with rows = 0 the counts, V and the overlap are 0 and the layer pointers are not
+ * read (they may be NULL, as an empty tensor's are).
  * workspace: >= DSA_WS_HEADER_BYTES bytes. n_keys <= 1,500,000 (larger: DSA_ERR_UNSUPPORTED).
  * -------------------------------------------------------------------------------------*/
 DSA_API dsa_status topk_overlap(const int32_t* const* layer_idx, int32_t n_layers, int32_t rows,

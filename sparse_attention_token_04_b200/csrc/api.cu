@@ -333,7 +333,7 @@ DSA_API dsa_status topk_overlap(const int32_t* const* layer_idx, int32_t n_layer
   if (n_keys > 1500000) return DSA_ERR_UNSUPPORTED;
   if (workspace_bytes < DSA_WS_HEADER_BYTES || !aligned(workspace, 256)) return DSA_ERR_INVALID;
   for (int i = 0; i < n_layers; ++i)
-    if (!layer_idx[i]) return DSA_ERR_INVALID;
+    if (!layer_idx[i] && rows > 0) return DSA_ERR_INVALID;  // zero rows read no layer
   const int sms = current_num_sms();
   if (sms < 1) return DSA_ERR_CUDA;
   return launch_overlap(layer_idx, n_layers, rows, topk, n_keys, out_counts, out_valid, out_overlap,
