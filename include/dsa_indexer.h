@@ -261,7 +261,8 @@ DSA_API dsa_status indexcache_run_lagged(const char* pattern, int32_t n_layers,
  *          i32 index rows as the indexer writes them (distinct entries in [0, n_keys), -1
  *          padding). Pointers may repeat (aliased S layers).
  * out_counts [n_layers][n_layers] u64: C[i][j] = sum over rows of |T_i(row) ∩ T_j(row)|.
- * out_valid  [1] u64: V = number of non-negative entries of layer 0.
+ * out_valid  [1] u64: V = number of non-negative entries of layer 0 (= C[0][0], since a row lists a
+ *          key at most once).
  * out_overlap [n_layers][n_layers] f64 = C / V, or NULL.
  * An entry outside [-1, n_keys) is skipped and recorded as DSA_ERR_DEVICE.
  * rows >= 0; with rows = 0 the counts, V and the overlap are 0 and the layer pointers are not

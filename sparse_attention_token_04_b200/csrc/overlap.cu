@@ -46,7 +46,7 @@ __global__ void __launch_bounds__(kOverlapThreads, kOverlapMinBlocks)
     overlap_bitmaps_kernel(const __grid_constant__ OverlapParams p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const int N = p.N;
-  // Pair counters (SMALL: the kOvGroup x kOvGroup triangle, whatever N), then the valid count.
+  // Pair counters (SMALL: the kOvGroup x kOvGroup triangle, whatever N), then one spare word.
   const int npairs = SMALL ? kOvPairs : N * (N + 1) / 2;
   unsigned long long* acc = overlap_acc(smem_raw);                        // [npairs + 1]
   int* row_max = reinterpret_cast<int*>(acc + npairs + 1);                 // [1] (+pad)
@@ -77,7 +77,6 @@ __global__ void __launch_bounds__(kOverlapThreads, kOverlapMinBlocks)
   for (int row = blockIdx.x; row < p.rows; row += gridDim.x) {
     const size_t off = static_cast<size_t>(row) * p.topk;
     int local_max = -1;
-    uint32_t valid0 = 0;
     for (int i = 0; i < N; ++i) {
       int32_t v[kOvPerThread];
       if constexpr (VEC) {
@@ -103,9 +102,8 @@ __global__ void __launch_bounds__(kOverlapThreads, kOverlapMinBlocks)
       for (int q = 0; q < kOvPerThread; ++q) {
         const int32_t x = v[q];
         if (x >= 0 && x < p.n_keys) {
-          atomicOr(&bi[x >> 5], 1u << (x & 31));
+          atomicOr(&bi[x >> 5], __funnelshift_l(0u, 1u, static_cast<uint32_t>(x)));  // 1 << (x mod 32)
           local_max = x > local_max ? x : local_max;
-          if (i == 0) ++valid0;
         } else if (x != -1) {
           record_error(p.hdr, DSA_ERR_DEVICE, DETAIL_BAD_INDEX);
         }
@@ -113,8 +111,6 @@ __global__ void __launch_bounds__(kOverlapThreads, kOverlapMinBlocks)
     }
     local_max = __reduce_max_sync(0xFFFFFFFFu, local_max);  // one shared atomic per warp
     if (lane == 0 && local_max >= 0) atomicMax(row_max, local_max);
-    valid0 = __reduce_add_sync(0xFFFFFFFFu, valid0);
-    if (lane == 0 && valid0) atomicAdd(&acc[npairs], static_cast<unsigned long long>(valid0));
     __syncthreads();
     const int wr = (*row_max >> 5) + 1;  // words that can hold a mark in this row
     if constexpr (SMALL) {
@@ -163,7 +159,8 @@ __global__ void __launch_bounds__(kOverlapThreads, kOverlapMinBlocks)
       for (int i = 0; i < kOvGroup; ++i)
         for (int j = i; j < kOvGroup; ++j, ++q)
           if (j < N && acc[q]) atomicAdd(&p.counts[i * N + j], acc[q]);
-      if (acc[npairs]) atomicAdd(p.valid, acc[npairs]);
+      // V: a row lists a key once, so layer 0's in-range entries are its pair count C[0][0].
+      if (acc[0]) atomicAdd(p.valid, acc[0]);
     }
   } else {
     __syncthreads();
@@ -171,7 +168,7 @@ __global__ void __launch_bounds__(kOverlapThreads, kOverlapMinBlocks)
     for (int i = 0; i < N; ++i)
       for (int j = i; j < N; ++j, ++pair)
         if (threadIdx.x == 0 && acc[pair]) atomicAdd(&p.counts[i * N + j], acc[pair]);
-    if (threadIdx.x == 0 && acc[npairs]) atomicAdd(p.valid, acc[npairs]);
+    if (threadIdx.x == 0 && acc[0]) atomicAdd(p.valid, acc[0]);  // V = C[0][0]
   }
 }
 
