@@ -93,7 +93,7 @@ size_t decode_workspace_bytes(int B, int max_len, int H, int d, int topk);
 // the per-request score histograms [B][kDecodeScoreBins] u32, the per-request collection state
 // [B][4] u32 (candidate count, largest ordered score, complement of the smallest, candidate
 // count the histogram predicts) and the per-request candidate keys [B][kDecodeCandCap] u64.
-// Histograms and state are adjacent so that one memset clears both.
+// Histograms and state are adjacent so that one small kernel (decode_clear_kernel) clears both.
 constexpr int kDecodeScoreBins = 2048;
 constexpr uint32_t kDecodeCandCap = 8192;
 struct DecodeLayout {
