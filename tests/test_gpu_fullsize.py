@@ -110,7 +110,7 @@ def test_decode_32_requests_47_layers_searched_pattern():
     for l in range(47):
         assert ptrs[l] == buf_of[src[l]].data_ptr()
     table_h, seq_h = table.cpu().numpy(), seq.cpu().numpy()
-    for l in (f_layers[0], f_layers[-1]):
+    for l in (f_layers[0], f_layers[4], f_layers[8], f_layers[-1]):  # all 32 requests of 4 F layers
         gpu = buf_of[l].cpu().numpy()
         ref = O.decode_rows(layers[l].numpy(), table_h, seq_h, topk)
         for b, r in enumerate(ref):
@@ -153,7 +153,7 @@ def test_prefill_200k_47_layers_searched_pattern_chunk_major():
     torch.cuda.synchronize()
     assert B.dsa_read_device_status(ws) == (0, 0)
     for n, l in enumerate((f_layers[0], f_layers[len(f_layers) // 2], f_layers[-1])):
-        rows = _boundary_rows(L, topk, chunk, 8, seed=500 + n)
+        rows = _boundary_rows(L, topk, chunk, 24, seed=500 + n)  # 43 rows per layer, 129 in all
         host_k = (layers[l].k.cpu().numpy(), layers[l].k_scale.cpu().numpy())
         gpu = full[l][torch.tensor(rows, device="cuda")].cpu().numpy()
         for i, t in enumerate(rows):

@@ -57,7 +57,7 @@ def test_long_context_gmm_keys_chunked():
     (cluster std 0.5), q ~ N(0, 1), w ~ N(0, 1)/8; 16 chunks of 8192 queries."""
     L, topk = 131072, 2048
     layer = gmm_layer(L, 64, 128, seed=3, device="cuda")
-    rows = boundary_rows(L, topk, 40, seed=31)
+    rows = boundary_rows(L, topk, 248, seed=31)  # 256 rows over all 16 chunks
     gpu = chunked_rows(layer, topk, rows)
     check_against_oracle(layer, topk, rows, gpu)
 
