@@ -356,13 +356,13 @@ dsa_status launch_prefill_sample_threshold(const uint64_t* cand, const uint32_t*
 }
 
 // Decode collection: CTA (c, b) takes scores [c * kCollectChunk, (c + 1) * kCollectChunk) of
-// request b. Four bulk copies bring its scores into shared memory while the CTA finds the
+// request b. Two bulk copies bring its scores into shared memory while the CTA finds the
 // request's boundary bin from the histogram: the highest bin at or above which at least k
 // scores lie (bin 0 when the request has at most k keys: every key is a winner). The keys at or
 // above that bin are appended to the request's candidate list, with one atomic reservation per
 // CTA, and the CTA's ordered score range is merged into the request's state (two more atomics).
 constexpr int kCollectThreads = 512;
-constexpr int kCollectParts = 4;
+constexpr int kCollectParts = 2;
 constexpr int kCollectPart = 4096;  // scores per bulk copy
 constexpr int kCollectChunk = kCollectParts * kCollectPart;
 static_assert(kDecodeScoreBins == 4 * kCollectThreads, "four histogram bins per thread");

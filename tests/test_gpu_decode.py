@@ -23,8 +23,8 @@ def run_decode(table, lens, layer, topk):
 @pytest.mark.parametrize("lens,topk", [([1, 63, 64, 65, 200, 3000, 2048, 2049], 2048),
                                        ([5000, 777, 130], 100), ([12000, 9000], 2048),
                                        # more tiles than resident scoring CTAs: ranges that
-                                       # cross requests, and requests over one 16384-score
-                                       # collection slice
+                                       # cross requests, and requests over several
+                                       # 8192-score collection slices
                                        (decode_lengths(48, 1000, 24000, seed=11), 2048),
                                        # many short requests: several request switches per CTA
                                        (decode_lengths(200, 100, 2000, seed=12), 64)])
