@@ -67,6 +67,36 @@ def test_lagged_prefill_consumers_read_previous_indexer_layer(keep_all):
         check_row(got[r.t], None, r, topk)
 
 
+def test_lagged_prefill_on_a_chunk():
+    """A chunk of queries [c0, L) against keys [0, L) (q_pos0 = c0): every consumer copy equals
+    the plain chunk call of its source layer, and a source layer's rows match the oracle."""
+    L, c0, topk, pattern = 1200, 700, 256, "FSFFS"
+    layers = [l.to("cuda") for l in correlated_layers(L, 64, 128, len(pattern), seed=21)]
+    chunk = [{"q": l.q[c0:], "q_scale": l.q_scale[c0:], "w": l.w[c0:], "k": l.k, "k_scale": l.k_scale}
+             for l in layers]
+    inputs = [d if c == "F" else None for d, c in zip(chunk, pattern)]
+    side = torch.cuda.Stream()
+    f_bufs = [torch.empty(L - c0, topk, dtype=torch.int32, device="cuda") for _ in range(2)]
+    by_ptr = {b.data_ptr(): b for b in f_bufs}
+    copies = {}
+    B.indexcache_run_lagged(pattern, inputs, topk, side, f_bufs=f_bufs, q_pos0=c0,
+                            consume=lambda l, p: copies.__setitem__(l, by_ptr[p].clone()))
+    torch.cuda.synchronize()
+    src = lagged_sources(pattern)
+    assert src == [0, 0, 0, 2, 3]
+    for l in sorted(set(src)):
+        ref, _ = B.dsa_indexer_prefill(chunk[l]["q"], chunk[l]["q_scale"], chunk[l]["w"], chunk[l]["k"],
+                                       chunk[l]["k_scale"], topk, q_pos0=c0, want_score=False)
+        torch.cuda.synchronize()
+        for j in range(len(pattern)):
+            if src[j] == l:
+                assert torch.equal(copies[j], ref), (j, l)
+    host = layers[2].numpy()
+    got = copies[3].cpu().numpy()
+    for r in O.prefill_rows(host, topk, [c0, c0 + 1, 900, L - 1]):
+        check_row(got[r.t - c0], None, r, topk)
+
+
 def test_lagged_decode_searched_pattern():
     lens = [5000, 300, 12000, 2049]
     topk, pattern = 512, SEARCHED_QUARTER_PATTERN
