@@ -20,5 +20,7 @@ from .inputs import (  # noqa: F401
     periodic_stream_layer,
     decode_lengths,
     paged_decode_layers,
+    LatentDecodeInputs,
+    latent_decode_inputs,
     SEARCHED_QUARTER_PATTERN,
 )

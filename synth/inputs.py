@@ -317,3 +317,41 @@ def paged_decode_layers(lens: Sequence[int], H: int, d: int, n_layers: int, seed
                               ks.reshape(nblk, block_size).contiguous())
 
     return table.to(device), seq_lens.to(device), layers()
+
+
+@dataclass
+class LatentDecodeInputs:
+    """Inputs of the sparse-attention consumer for one decode step: bf16 queries q[B][Hq][dqk],
+    a bf16 latent cache latent[n_blocks * block_size][dqk] laid out in the same physical blocks
+    as `block_table`, and selected logical positions idx[B][topk] (-1: none)."""
+    q: torch.Tensor
+    latent: torch.Tensor
+    block_table: torch.Tensor
+    seq_lens: torch.Tensor
+    idx: torch.Tensor
+
+
+def latent_decode_inputs(lens: Sequence[int], topk: int, seed: int, Hq: int = 128, dqk: int = 576,
+                         block_size: int = 64, device="cpu") -> LatentDecodeInputs:
+    """Random bf16 queries and latents (N(0, 1) rounded to bf16), a random block table as in
+    `paged_decode_layers`, and per request min(topk, len) distinct positions drawn uniformly
+    from [0, len) in random order, padded with -1."""
+    B = len(lens)
+    nb = [(int(n) + block_size - 1) // block_size for n in lens]
+    nblk = sum(nb)
+    g = _generator(seed, "cpu")
+    perm = torch.randperm(nblk, generator=g).to(torch.int32)
+    table = torch.full((B, max(1, max(nb) if nb else 1)), -1, dtype=torch.int32)
+    off = 0
+    for b in range(B):
+        table[b, :nb[b]] = perm[off:off + nb[b]]
+        off += nb[b]
+    idx = torch.full((B, topk), -1, dtype=torch.int32)
+    for b, n in enumerate(lens):
+        m = min(topk, int(n))
+        idx[b, :m] = torch.randperm(int(n), generator=g)[:m].to(torch.int32)
+    gd = _generator(seed + 1, device)
+    q = torch.randn(B, Hq, dqk, generator=gd, device=device).to(torch.bfloat16)
+    latent = torch.randn(nblk * block_size, dqk, generator=gd, device=device).to(torch.bfloat16)
+    seq = torch.tensor([int(n) for n in lens], dtype=torch.int32)
+    return LatentDecodeInputs(q, latent, table.to(device), seq.to(device), idx.to(device))
