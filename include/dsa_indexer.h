@@ -254,6 +254,37 @@ DSA_API dsa_status indexcache_run_lagged(const char* pattern, int32_t n_layers,
                                          size_t workspace_bytes, void* stream, void* indexer_stream);
 
 /* ---------------------------------------------------------------------------------------
+ * Sparse attention over the selected latents ("Index Share逻辑详解" §2: after the indexer's
+ * top-k selection, the core MLA attention runs on only those k latents). A consumer of the
+ * decode index buffer: one query per request with Hq = 128 heads over a dqk = 576-wide bf16
+ * latent cache whose first dv = 512 entries are the values. For request b and head h,
+ *     out[b][h] = sum_s softmax_s(scale * q[b][h] . K[s]) V[s],  K[s] = latent[row(b, s)],
+ *     V[s] = K[s][0:512],  row(b, s) = block_table[b][s / block_size] * block_size + s % block_size,
+ * over the logical positions s = idx[b][0..topk) (entries -1 select nothing; a request that
+ * selects nothing gets zeros).
+ *   q           [B][128][576]                    bf16 (as uint16), 16-byte aligned
+ *   latent      [n_blocks * block_size][576]     bf16, 16-byte aligned (the paged cache's rows)
+ *   block_table [B][max_blocks] i32, seq_lens [B] i32 (positions >= seq_lens[b] are invalid)
+ *   idx         [B][topk] i32 logical positions, as dsa_indexer_decode writes them
+ *   out         [B][128][512] f32, 16-byte aligned
+ * topk must be a multiple of 256, at most 2048; scale > 0. Products run on the tensor cores in
+ * bf16 with fp32 accumulation; the softmax weights are rounded to bf16 before the value product
+ * (their sum is taken over the rounded weights). A position outside [0, seq_lens[b]) other than
+ * -1, a bad length or a block-table entry outside [0, n_blocks) is recorded as DSA_ERR_DEVICE
+ * and the key is left out.
+ * workspace: >= dsa_sparse_attention_workspace_bytes(B, topk) bytes, 256-byte aligned.
+ * -------------------------------------------------------------------------------------*/
+DSA_API size_t dsa_sparse_attention_workspace_bytes(int32_t B, int32_t topk);
+
+DSA_API dsa_status dsa_sparse_attention_decode(const uint16_t* q, const uint16_t* latent,
+                                               int32_t n_blocks, int32_t block_size,
+                                               const int32_t* block_table, int32_t max_blocks,
+                                               const int32_t* seq_lens, const int32_t* idx,
+                                               int32_t B, int32_t Hq, int32_t dqk, int32_t dv,
+                                               int32_t topk, float scale, float* out,
+                                               void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------
  * Cross-layer top-k overlap ("IndexShare deep-dive report" §1.2: the overlap of layers i
  * and j is |T(i) ∩ T(j)| / k; adjacent layers overlap 70-100% in blocks).
  *

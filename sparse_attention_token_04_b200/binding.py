@@ -71,6 +71,9 @@ _SIGNATURES = {
     "dsa_topk_merge": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp]),
     "dsa_indexer_decode_noalloc": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _i32, _vp, _i32,
                                           _i32, _i32, _i32, _vp, _vp, _vp, _vp]),
+    "dsa_sparse_attention_workspace_bytes": (_sz, [_i32, _i32]),
+    "dsa_sparse_attention_decode": (_i32, [_vp, _vp, _i32, _i32, _vp, _i32, _vp, _vp, _i32, _i32, _i32,
+                                           _i32, _i32, ctypes.c_float, _vp, _vp, _sz, _vp]),
 }
 
 _LIB: Optional[ctypes.CDLL] = None
@@ -450,3 +453,35 @@ def dsa_indexer_decode_noalloc(q, q_scale, w, k_cache, k_scale_cache, block_tabl
                                             _ptr(device_status), _stream(stream)),
            "dsa_indexer_decode_noalloc")
     return out_idx, out_score
+
+
+def dsa_sparse_attention_workspace_bytes(B: int, topk: int) -> int:
+    return int(lib().dsa_sparse_attention_workspace_bytes(B, topk))
+
+
+def dsa_sparse_attention_decode(q, latent, block_table, seq_lens, idx, scale: float, block_size: int = 64,
+                                out=None, workspace=None, stream=None):
+    """Sparse attention of decode queries over their selected latents: q[B][128][576] bf16,
+    latent[n_blocks * block_size][576] bf16, block_table[B][max_blocks] i32, seq_lens[B] i32,
+    idx[B][topk] i32 -> out[B][128][512] f32."""
+    B, Hq, dqk = (int(x) for x in q.shape)
+    n_rows = int(latent.shape[0])
+    topk = int(idx.shape[1])
+    _need(q, "q", torch.bfloat16)
+    _need(latent, "latent", torch.bfloat16, (n_rows, dqk))
+    _need(block_table, "block_table", torch.int32)
+    _need(seq_lens, "seq_lens", torch.int32, (B,))
+    _need(idx, "idx", torch.int32, (B, topk))
+    if n_rows % block_size:
+        raise ValueError("latent rows must be whole blocks")
+    dv = 512
+    if out is None:
+        out = torch.empty(B, Hq, dv, dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.float32, (B, Hq, dv))
+    ws = _workspace(dsa_sparse_attention_workspace_bytes(B, topk), q.device, workspace, stream)
+    _check(lib().dsa_sparse_attention_decode(_ptr(q), _ptr(latent), n_rows // block_size, block_size,
+                                             _ptr(block_table), int(block_table.shape[1]), _ptr(seq_lens),
+                                             _ptr(idx), B, Hq, dqk, dv, topk, float(scale), _ptr(out),
+                                             _ptr(ws), ws.numel(), _stream(stream)),
+           "dsa_sparse_attention_decode")
+    return out

@@ -20,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(ROOT, "_build")
 LIB_PATH = os.path.join(PKG, "libdsa_indexer.so")
-SOURCES = ["api.cu", "prefill.cu", "decode.cu", "topk.cu", "overlap.cu", "selftest.cu", "noalloc.cu", "merge.cu", "pattern.cu"]
+SOURCES = ["api.cu", "prefill.cu", "decode.cu", "topk.cu", "overlap.cu", "selftest.cu", "noalloc.cu", "merge.cu", "pattern.cu", "attention.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ARCH + ["-lineinfo", "-O3", "-std=c++17", "-Xcompiler", "-fPIC,-fvisibility=hidden",
                 "-I", INCLUDE]

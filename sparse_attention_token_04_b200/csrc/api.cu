@@ -173,6 +173,35 @@ DSA_API dsa_status dsa_indexer_decode(const uint8_t* q, const float* q_scale, co
   return launch_decode(a);
 }
 
+DSA_API size_t dsa_sparse_attention_workspace_bytes(int32_t B, int32_t topk) {
+  if (B < 1 || topk < 256 || topk > DSA_MAX_TOPK || topk % 256 != 0) return 0;
+  return attention_workspace_bytes(B, topk);
+}
+
+DSA_API dsa_status dsa_sparse_attention_decode(const uint16_t* q, const uint16_t* latent,
+                                               int32_t n_blocks, int32_t block_size,
+                                               const int32_t* block_table, int32_t max_blocks,
+                                               const int32_t* seq_lens, const int32_t* idx,
+                                               int32_t B, int32_t Hq, int32_t dqk, int32_t dv,
+                                               int32_t topk, float scale, float* out,
+                                               void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !latent || !block_table || !seq_lens || !idx || !out) return DSA_ERR_INVALID;
+  if (B < 1 || n_blocks < 1 || block_size < 1 || max_blocks < 1 || topk < 1) return DSA_ERR_INVALID;
+  if (static_cast<int64_t>(max_blocks) * block_size > INT32_MAX ||
+      static_cast<int64_t>(n_blocks) * block_size > INT32_MAX)
+    return DSA_ERR_INVALID;
+  if (!(scale > 0.0f) || !(scale < 1e30f)) return DSA_ERR_INVALID;
+  if (!aligned(q, 16) || !aligned(latent, 16) || !aligned(out, 16)) return DSA_ERR_INVALID;
+  if (Hq != 128 || dqk != 576 || dv != 512 || topk % 256 != 0 || topk > DSA_MAX_TOPK ||
+      B > DSA_DECODE_MAX_REQUESTS)
+    return DSA_ERR_UNSUPPORTED;
+  if (!workspace || !aligned(workspace, 256)) return DSA_ERR_INVALID;
+  if (workspace_bytes < attention_workspace_bytes(B, topk)) return DSA_ERR_INVALID;
+  AttentionLaunch a{q, latent, n_blocks, block_size, block_table, max_blocks, seq_lens, idx, B, topk,
+                    scale, out, workspace, static_cast<cudaStream_t>(stream), wait_budget_ns()};
+  return launch_attention(a);
+}
+
 DSA_API size_t dsa_indexcache_workspace_bytes(const dsa_indexer_shape* shape) {
   if (!shape) return 0;
   if (shape->mode == DSA_MODE_PREFILL)

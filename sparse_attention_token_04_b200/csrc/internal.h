@@ -46,6 +46,22 @@ struct DecodeLaunch {
   int num_sms;
 };
 
+struct AttentionLaunch {
+  const uint16_t* q;
+  const uint16_t* latent;
+  int32_t n_blocks, block_size;
+  const int32_t* block_table;
+  int32_t max_blocks;
+  const int32_t* seq_lens;
+  const int32_t* idx;
+  int32_t B, topk;
+  float scale;
+  float* out;
+  void* ws;
+  cudaStream_t stream;
+  uint64_t budget_ns;
+};
+
 // Prefill workspace layout. Every query row owns 4 * seg_stride candidate entries: four warp
 // segments, seg_stride entries apart. The lean pass may fill a segment up to lean_segcap
 // (about 3k/4 + 128: it expects k + 6.5 sqrt(k S) keys per row), the exact pass up to
@@ -129,6 +145,9 @@ dsa_status launch_decode(const DecodeLaunch& a);
 dsa_status launch_decode_topk(void* ws, const DecodeLayout& lay, int max_len,
                               const int32_t* seq_lens, int B, int topk, int32_t* out_idx,
                               float* out_score, uint64_t budget_ns, cudaStream_t stream);
+// Sparse attention of decode queries over their selected latents (attention.cu).
+size_t attention_workspace_bytes(int B, int topk);
+dsa_status launch_attention(const AttentionLaunch& a);
 dsa_status launch_overlap(const int32_t* const* layer_idx, int32_t n_layers, int32_t rows,
                           int32_t topk, int32_t n_keys, uint64_t* out_counts, uint64_t* out_valid,
                           double* out_overlap, void* ws, cudaStream_t stream, int num_sms);
