@@ -552,14 +552,14 @@ def run_decode(args, world, rank, device, peaks):
             "gpu_launches": DECODE_LAUNCHES_PER_CALL * n_full * args.decode_steps}
 
 
-def run_mli_decode(args, world, rank, device):
-    """The 47-layer decode step with a consumer on every layer, under plain IndexCache and under
-    the lagged multi-layer-indexer mode at the same retention (searched 1/4 pattern). The consumer
-    stands in for the model's sparse attention: it gathers every request's selected rows of a
-    576-wide bf16 latent cache (one cache shared by all layers) and runs softmax(q K^T) V for 128
-    query heads with PyTorch ops on the consumer stream. Plain: each layer's consumer follows its
-    own indexer on one stream. Lagged: every Full layer's indexer runs on a second stream while
-    the consumers read the previous indexer layer's selection."""
+def run_mli_decode(args, world, rank, device, peaks):
+    """The 47-layer decode step with the sparse-attention consumer on every layer, under plain
+    IndexCache and under the lagged multi-layer-indexer mode at the same retention (searched 1/4
+    pattern). The consumer is dsa_sparse_attention_decode: 128 query heads over the 2048 selected
+    rows of a 576-wide bf16 latent cache (one cache shared by all layers, the indexer's paged
+    layout), values the first 512 entries. Plain: each layer's consumer follows its own indexer on
+    one stream. Lagged: every Full layer's indexer runs on a second stream while the consumers read
+    the previous indexer layer's selection. The consumer alone is also timed, with its roofline."""
     from sparse_attention_token_04_b200 import binding as B
     from synth import SEARCHED_QUARTER_PATTERN, decode_lengths, paged_decode_layers
 
@@ -583,17 +583,15 @@ def run_mli_decode(args, world, rank, device):
     ws = torch.empty(B.dsa_decode_workspace_bytes(Bn, table.shape[1] * 64, cfg["H"], cfg["d"], topk),
                      dtype=torch.uint8, device=device)
     B.dsa_workspace_init(ws)
+    att_ws = torch.empty(B.dsa_sparse_attention_workspace_bytes(Bn, topk), dtype=torch.uint8, device=device)
+    B.dsa_workspace_init(att_ws)
+    att_out = torch.empty(Bn, heads, dv, dtype=torch.float32, device=device)
     side = torch.cuda.Stream(device=device)
     stream = torch.cuda.current_stream()
 
     def consume(l, ptr):
-        idx = by_ptr[ptr].long()
-        valid = idx >= 0
-        phys = table.long().gather(1, (idx.clamp(min=0) // 64)) * 64 + idx.clamp(min=0) % 64
-        kv = latent.index_select(0, phys.view(-1)).view(Bn, topk, dkv)
-        sc = torch.bmm(q_att, kv.transpose(1, 2)).float() * scale
-        sc.masked_fill_(~valid[:, None, :], float("-inf"))
-        torch.bmm(torch.softmax(sc, dim=-1).to(torch.bfloat16), kv[..., :dv])
+        B.dsa_sparse_attention_decode(q_att, latent, table, seq, by_ptr[ptr], scale, out=att_out,
+                                      workspace=att_ws)
 
     def plain():
         B.indexcache_run(pattern, inputs, topk, mode=B.DSA_MODE_DECODE, f_bufs=bufs[:1],
@@ -613,15 +611,28 @@ def run_mli_decode(args, world, rank, device):
             fn()
         torch.cuda.synchronize()
         res[name] = timed(stream, fn, args.mli_steps) / args.mli_steps
-    if B.dsa_read_device_status(ws) != (0, 0):
+    if B.dsa_read_device_status(ws) != (0, 0) or B.dsa_read_device_status(att_ws) != (0, 0):
         raise RuntimeError("device status after the lagged decode steps")
+    call_ms = res["consumers_only"] / len(pattern)
+    att_bytes = Bn * topk * dkv * 2 + Bn * heads * dkv * 2 + Bn * heads * dv * 4 + Bn * topk * 4
+    att_flop = 2.0 * Bn * heads * topk * (dkv + dv)
+    gbs = att_bytes / (call_ms / 1e3) / 1e9
+    tflops = att_flop / (call_ms / 1e3) / 1e12
+    bf16_peak = float(peaks["bf16_tflops"])
     return {"workload": "47-layer decode step, 32 requests U[10000,200000], searched 1/4 pattern (12 "
-                        "indexer layers), a sparse-attention stand-in consumer on every layer (gather of "
-                        "the 2048 selected rows of a 576-wide bf16 latent cache, softmax(qK^T)V for 128 "
-                        "heads, PyTorch ops)",
+                        "indexer layers), the sparse-attention consumer (dsa_sparse_attention_decode: 128 "
+                        "heads over the 2048 selected rows of a 576-wide bf16 latent cache) on every layer",
             "plain_indexcache_ms": res["plain"], "lagged_mli_ms": res["lagged"],
             "consumers_alone_ms": res["consumers_only"],
-            "speedup_lagged_vs_plain": res["plain"] / res["lagged"], "steps": args.mli_steps}
+            "speedup_lagged_vs_plain": res["plain"] / res["lagged"], "steps": args.mli_steps,
+            "attention_call": {
+                "kernel": "attention_split_kernel + attention_combine_kernel",
+                "launch_ms": call_ms, "bound": "hbm",
+                "algorithmic_per_launch": f"{att_bytes} B (2048 selected 1152-byte latent rows per request, "
+                                          f"q, out, indices); {att_flop:.4e} FLOP",
+                "achieved": gbs, "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                "frac": gbs / float(peaks["hbm_gbs"]),
+                "tflops": tflops, "tflops_frac_of_bf16_burst": tflops / bf16_peak}}
 
 
 # DRAM bytes (read + write) per cached key of decode_indexer_kernel from one ncu capture of this
@@ -717,7 +728,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.empty_cache()
     stack = run_stack16k(args, world, rank, device, peaks, peak_kind) if args.stack_steps > 0 else None
     decode = run_decode(args, world, rank, device, peaks) if args.decode_steps > 0 else None
-    mli = run_mli_decode(args, world, rank, device) if args.mli_steps > 0 else None
+    mli = run_mli_decode(args, world, rank, device, peaks) if args.mli_steps > 0 else None
 
     if rank == 0:
         c = LONG
