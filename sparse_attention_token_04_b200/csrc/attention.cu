@@ -12,8 +12,9 @@
 // in shared memory with the 128-byte swizzle, written by the CTA's threads (cp.async for the
 // query and key rows, register transposes for the values), and every product runs on the
 // tensor cores (tcgen05.mma kind::f16, FP32 accumulators in TMEM):
-//   1. S[128 heads][256 keys] = Q . K^T over the 576 dims, nine 64-dim chunks double-buffered
-//      (each chunk: four M=128, N=256, K=16 MMAs into TMEM columns 0..255);
+//   1. S[128 heads][256 keys] = Q . K^T over the 576 dims, nine 64-dim chunks in three stages,
+//      loaded two chunks ahead (each chunk: four M=128, N=256, K=16 MMAs into TMEM columns
+//      0..255);
 //   2. four warps (thread = head) read S, mask unselected keys, and form the split's softmax
 //      numerators P = exp(scale (S - m)) in bf16 (shared memory, K-major) with the row max m
 //      and sum l in fp32;
@@ -42,14 +43,16 @@ constexpr int kAttThreads = 256;
 constexpr int kAttQkChunks = kAttDqk / kAttChunk;   // 9
 constexpr int kAttPvChunks = kAttSplit / kAttChunk;  // 4
 
+constexpr int kAttQkStages = 3;
+
 struct AttSmem {
-  // QK stages: Q chunk [128][64] + K chunk [256][64] bf16 each (48 KB); the V^T stages
+  // QK stages: Q chunk [128][64] + K chunk [256][64] bf16 each (48 KB); the two V^T stages
   // [256 dims][64 keys] (32 KB each) reuse them once S is complete.
-  uint8_t stage[2][48 * 1024];
+  uint8_t stage[kAttQkStages][48 * 1024];
   uint8_t p[kAttPvChunks][kAttHeads * 128];  // P [128 heads][256 keys] as four K-major 64-key chunks
   int32_t rows[kAttSplit];                   // latent row of each selected key, -1: masked
   float m[kAttHeads], l[kAttHeads];
-  uint64_t qk_done[2], pv_done[2];
+  uint64_t qk_done[kAttQkStages], pv_done[2];
   uint32_t tmem;
   int abort;
 };
@@ -109,10 +112,8 @@ __global__ void __launch_bounds__(kAttThreads, 1) attention_split_kernel(const _
   const int c = blockIdx.x, v = blockIdx.y, b = blockIdx.z;
   const int n_split = gridDim.x;
   if (tid == 0) {
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sm.qk_done[i], 1);
-      mbar_init(&sm.pv_done[i], 1);
-    }
+    for (int i = 0; i < kAttQkStages; ++i) mbar_init(&sm.qk_done[i], 1);
+    for (int i = 0; i < 2; ++i) mbar_init(&sm.pv_done[i], 1);
     fence_mbar_init();
     sm.abort = 0;
   }
@@ -146,13 +147,11 @@ __global__ void __launch_bounds__(kAttThreads, 1) attention_split_kernel(const _
   const WaitCtl ctl{p.hdr, &sm.abort, p.budget_ns};
   const uint16_t* qb = p.q + static_cast<size_t>(b) * kAttHeads * kAttDqk;
   bool ok = true;
-  uint32_t qk_issued[2] = {0, 0}, pv_issued[2] = {0, 0};
+  uint32_t qk_issued[kAttQkStages] = {0, 0, 0}, pv_issued[2] = {0, 0};
 
-  // 1. S = Q K^T over nine 64-dim chunks.
-  for (int ch = 0; ch < kAttQkChunks && ok; ++ch) {
-    const int st = ch & 1;
-    if (qk_issued[st] > 0) ok = mbar_wait(&sm.qk_done[st], (qk_issued[st] - 1) & 1u, ctl, DETAIL_WAIT_ACCFULL);
-    if (__syncthreads_or(!ok)) { ok = false; break; }
+  // 1. S = Q K^T over nine 64-dim chunks, loads two chunks ahead of the MMAs (three stages).
+  auto load_qk = [&](int ch) {
+    const int st = ch % kAttQkStages;
     uint8_t* qs = sm.stage[st];
     uint8_t* ks = sm.stage[st] + kAttHeads * 128;
 #pragma unroll
@@ -168,12 +167,29 @@ __global__ void __launch_bounds__(kAttThreads, 1) attention_split_kernel(const _
       cp_async_16(ks + sw128(r, j), src, row < 0 ? 0u : 16u);
     }
     cp_async_commit();
-    cp_async_wait<0>();
+  };
+  load_qk(0);
+  load_qk(1);
+  for (int ch = 0; ch < kAttQkChunks && ok; ++ch) {
+    const int st = ch % kAttQkStages;
+    if (ch + 2 < kAttQkChunks) {
+      // stage (ch + 2) % 3 was last read by the MMAs of chunk ch - 1
+      const int sn = (ch + 2) % kAttQkStages;
+      if (qk_issued[sn] > 0) ok = mbar_wait(&sm.qk_done[sn], (qk_issued[sn] - 1) & 1u, ctl, DETAIL_WAIT_ACCFULL);
+      if (__syncthreads_or(!ok)) { ok = false; break; }
+      load_qk(ch + 2);
+      cp_async_wait<2>();  // this thread's copies of chunk ch have landed
+    } else if (ch + 1 < kAttQkChunks) {
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
     fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
       tc_fence_after();
-      const uint64_t da = make_smem_desc(smem_u32(qs), 128), db = make_smem_desc(smem_u32(ks), 128);
+      const uint64_t da = make_smem_desc(smem_u32(sm.stage[st]), 128);
+      const uint64_t db = make_smem_desc(smem_u32(sm.stage[st] + kAttHeads * 128), 128);
 #pragma unroll
       for (int kk = 0; kk < kAttChunk / 16; ++kk)
         tc_mma_bf16(tS, da + 2ull * kk, db + 2ull * kk, make_idesc_bf16(kAttHeads, kAttSplit),
@@ -182,8 +198,9 @@ __global__ void __launch_bounds__(kAttThreads, 1) attention_split_kernel(const _
     }
     ++qk_issued[st];
   }
+  cp_async_wait<0>();  // nothing of this CTA's is still landing (also on the abort path)
   // S complete: the last chunk's commit covers every earlier MMA.
-  const int last_qk = (kAttQkChunks - 1) & 1;
+  const int last_qk = (kAttQkChunks - 1) % kAttQkStages;
   if (ok) ok = mbar_wait(&sm.qk_done[last_qk], (qk_issued[last_qk] - 1) & 1u, ctl, DETAIL_WAIT_ACCFULL);
   ok = !__syncthreads_or(!ok);
 
@@ -231,14 +248,10 @@ __global__ void __launch_bounds__(kAttThreads, 1) attention_split_kernel(const _
   fence_proxy_async_smem();
   __syncthreads();
 
-  // 3. O = P V over four 64-key chunks; V^T chunks are built by 8x8 register transposes.
+  // 3. O = P V over four 64-key chunks; V^T chunks are built by 8x8 register transposes, the
+  // next chunk's rows loading while the current one is transposed.
   const uint32_t ko = tid & 7u, dO = tid >> 3;  // key octet, dim octet (32 of them: 256 dims)
-  for (int kc = 0; kc < kAttPvChunks && ok; ++kc) {
-    const int st = kc & 1;
-    if (pv_issued[st] > 0) ok = mbar_wait(&sm.pv_done[st], (pv_issued[st] - 1) & 1u, ctl, DETAIL_WAIT_ACCFULL);
-    if (__syncthreads_or(!ok)) { ok = false; break; }
-    uint8_t* vt = sm.stage[st];  // [256 dims][64 keys]
-    uint4 x[8];
+  auto load_v = [&](int kc, uint4 (&x)[8]) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int row = sm.rows[kc * kAttChunk + ko * 8 + i];
@@ -246,8 +259,17 @@ __global__ void __launch_bounds__(kAttThreads, 1) attention_split_kernel(const _
                      : __ldg(reinterpret_cast<const uint4*>(p.latent + static_cast<size_t>(row) * kAttDqk +
                                                             v * kAttHalf + dO * 8));
     }
-    // x[i] holds dims dO*8 .. +7 of key i; out[e] gathers dim e of keys 0..7.
-    const uint32_t* xw = reinterpret_cast<const uint32_t*>(x);
+  };
+  uint4 xa[8], xb[8];
+  if (ok) load_v(0, xa);
+  for (int kc = 0; kc < kAttPvChunks && ok; ++kc) {
+    const int st = kc & 1;
+    if (pv_issued[st] > 0) ok = mbar_wait(&sm.pv_done[st], (pv_issued[st] - 1) & 1u, ctl, DETAIL_WAIT_ACCFULL);
+    if (__syncthreads_or(!ok)) { ok = false; break; }
+    if (kc + 1 < kAttPvChunks) load_v(kc + 1, xb);
+    uint8_t* vt = sm.stage[st];  // [256 dims][64 keys]
+    // xa[i] holds dims dO*8 .. +7 of key i; row e of the block gathers dim e of keys 0..7.
+    const uint32_t* xw = reinterpret_cast<const uint32_t*>(xa);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       uint32_t w[4];
@@ -270,6 +292,8 @@ __global__ void __launch_bounds__(kAttThreads, 1) attention_split_kernel(const _
       tc_commit(&sm.pv_done[st]);
     }
     ++pv_issued[st];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) xa[i] = xb[i];
   }
   const int last_pv = (kAttPvChunks - 1) & 1;
   if (ok) ok = mbar_wait(&sm.pv_done[last_pv], (pv_issued[last_pv] - 1) & 1u, ctl, DETAIL_WAIT_ACCFULL);
@@ -300,10 +324,10 @@ __global__ void __launch_bounds__(kAttThreads, 1) attention_split_kernel(const _
   }
   if (!ok && tid == 0) {
     // Let the MMAs this CTA issued land before its TMEM is freed (bounded).
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kAttQkStages; ++i)
       if (qk_issued[i]) mbar_wait_drain(&sm.qk_done[i], (qk_issued[i] - 1) & 1u, p.budget_ns);
+    for (int i = 0; i < 2; ++i)
       if (pv_issued[i]) mbar_wait_drain(&sm.pv_done[i], (pv_issued[i] - 1) & 1u, p.budget_ns);
-    }
   }
   __syncthreads();
   if (warp == 0) {
