@@ -7,8 +7,8 @@
 // values. For request b and head h:
 //     out[b, h] = sum_s softmax_s(scale * q[b, h] . K[s]) V[s]  over the selected positions s.
 //
-// attention_split_kernel: CTA (c, v, b) takes the 256 selected positions c*256 .. c*256+255 of
-// request b and the value half v (dims v*256 .. v*256+255). All operands are K-major bf16 tiles
+// attention_split_kernel: CTA (c, b) takes the 256 selected positions c*256 .. c*256+255 of
+// request b. All operands are K-major bf16 tiles
 // in shared memory with the 128-byte swizzle, written by the CTA's threads (cp.async for the
 // query and key rows, register transposes for the values), and every product runs on the
 // tensor cores (tcgen05.mma kind::f16, FP32 accumulators in TMEM):
@@ -18,9 +18,10 @@
 //   2. four warps (thread = head) read S, mask unselected keys, and form the split's softmax
 //      numerators P = exp(scale (S - m)) in bf16 (shared memory, K-major) with the row max m
 //      and sum l in fp32;
-//   3. O[128][256] = P . V over the 256 keys, four 64-key chunks whose V^T tiles are built by
-//      transposing 8x8 blocks in registers (MMAs into TMEM columns 256..511);
-//   4. O, m and l go to the workspace.
+//   3. for each value half (dims 0..255, then 256..511): O[128][256] = P . V over the 256 keys,
+//      four 64-key chunks whose V^T tiles are built by transposing 8x8 blocks in registers
+//      (MMAs into TMEM columns 256..511, which S no longer needs), and the half of O goes to the
+//      workspace; m and l go with the first half.
 // attention_combine_kernel then merges the splits of a request (log-sum-exp weights) into out.
 // Waits on the tensor core are bounded; a timeout is recorded as DSA_ERR_TIMEOUT.
 #include <algorithm>
@@ -109,7 +110,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attention_split_kernel(const _
   AttSmem& sm = *reinterpret_cast<AttSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
   const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
-  const int c = blockIdx.x, v = blockIdx.y, b = blockIdx.z;
+  const int c = blockIdx.x, b = blockIdx.z;
   const int n_split = gridDim.x;
   if (tid == 0) {
     for (int i = 0; i < kAttQkStages; ++i) mbar_init(&sm.qk_done[i], 1);
@@ -248,10 +249,11 @@ __global__ void __launch_bounds__(kAttThreads, 1) attention_split_kernel(const _
   fence_proxy_async_smem();
   __syncthreads();
 
-  // 3. O = P V over four 64-key chunks; V^T chunks are built by 8x8 register transposes, the
-  // next chunk's rows loading while the current one is transposed.
+  // 3. and 4., once per value half v: O = P V over four 64-key chunks into TMEM columns
+  // 256..511 (V^T chunks built by 8x8 register transposes, the next chunk's rows loading while
+  // the current one is transposed), then the unnormalised O of the half to the workspace.
   const uint32_t ko = tid & 7u, dO = tid >> 3;  // key octet, dim octet (32 of them: 256 dims)
-  auto load_v = [&](int kc, uint4 (&x)[8]) {
+  auto load_v = [&](int v, int kc, uint4 (&x)[8]) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int row = sm.rows[kc * kAttChunk + ko * 8 + i];
@@ -261,66 +263,67 @@ __global__ void __launch_bounds__(kAttThreads, 1) attention_split_kernel(const _
     }
   };
   uint4 xa[8], xb[8];
-  if (ok) load_v(0, xa);
-  for (int kc = 0; kc < kAttPvChunks && ok; ++kc) {
-    const int st = kc & 1;
-    if (pv_issued[st] > 0) ok = mbar_wait(&sm.pv_done[st], (pv_issued[st] - 1) & 1u, ctl, DETAIL_WAIT_ACCFULL);
-    if (__syncthreads_or(!ok)) { ok = false; break; }
-    if (kc + 1 < kAttPvChunks) load_v(kc + 1, xb);
-    uint8_t* vt = sm.stage[st];  // [256 dims][64 keys]
-    // xa[i] holds dims dO*8 .. +7 of key i; row e of the block gathers dim e of keys 0..7.
-    const uint32_t* xw = reinterpret_cast<const uint32_t*>(xa);
+  for (int v = 0; v < kAttDv / kAttHalf && ok; ++v) {
+    load_v(v, 0, xa);
+    for (int kc = 0; kc < kAttPvChunks && ok; ++kc) {
+      const int st = kc & 1;
+      if (pv_issued[st] > 0) ok = mbar_wait(&sm.pv_done[st], (pv_issued[st] - 1) & 1u, ctl, DETAIL_WAIT_ACCFULL);
+      if (__syncthreads_or(!ok)) { ok = false; break; }
+      if (kc + 1 < kAttPvChunks) load_v(v, kc + 1, xb);
+      uint8_t* vt = sm.stage[st];  // [256 dims][64 keys]
+      // xa[i] holds dims dO*8 .. +7 of key i; row e of the block gathers dim e of keys 0..7.
+      const uint32_t* xw = reinterpret_cast<const uint32_t*>(xa);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      uint32_t w[4];
+      for (int e = 0; e < 8; ++e) {
+        uint32_t w[4];
 #pragma unroll
-      for (int k2 = 0; k2 < 4; ++k2) {
-        const uint32_t a = xw[(2 * k2) * 4 + (e >> 1)], bb = xw[(2 * k2 + 1) * 4 + (e >> 1)];
-        w[k2] = __byte_perm(a, bb, (e & 1) ? 0x7632u : 0x5410u);
+        for (int k2 = 0; k2 < 4; ++k2) {
+          const uint32_t a = xw[(2 * k2) * 4 + (e >> 1)], bb = xw[(2 * k2 + 1) * 4 + (e >> 1)];
+          w[k2] = __byte_perm(a, bb, (e & 1) ? 0x7632u : 0x5410u);
+        }
+        *reinterpret_cast<uint4*>(vt + sw128(dO * 8 + e, ko)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
-      *reinterpret_cast<uint4*>(vt + sw128(dO * 8 + e, ko)) = make_uint4(w[0], w[1], w[2], w[3]);
+      fence_proxy_async_smem();
+      __syncthreads();
+      if (tid == 0) {
+        tc_fence_after();
+        const uint64_t da = make_smem_desc(smem_u32(sm.p[kc]), 128), db = make_smem_desc(smem_u32(vt), 128);
+#pragma unroll
+        for (int kk = 0; kk < kAttChunk / 16; ++kk)
+          tc_mma_bf16(tO, da + 2ull * kk, db + 2ull * kk, make_idesc_bf16(kAttHeads, kAttHalf),
+                      (kc > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&sm.pv_done[st]);
+      }
+      ++pv_issued[st];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) xa[i] = xb[i];
     }
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 0) {
+    const int last_pv = (kAttPvChunks - 1) & 1;
+    if (ok) ok = mbar_wait(&sm.pv_done[last_pv], (pv_issued[last_pv] - 1) & 1u, ctl, DETAIL_WAIT_ACCFULL);
+    ok = !__syncthreads_or(!ok);
+    if (ok && warp < 4) {
       tc_fence_after();
-      const uint64_t da = make_smem_desc(smem_u32(sm.p[kc]), 128), db = make_smem_desc(smem_u32(vt), 128);
+      const uint32_t h = warp * 32u + lane;
+      const uint32_t lane_base = (warp * 32u) << 16;
+      float* dst = p.o_part + ((static_cast<size_t>(b) * n_split + c) * kAttHeads + h) * kAttDv + v * kAttHalf;
+      for (int cc = 0; cc < kAttHalf / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tO + lane_base + cc * 32, r);
+        tmem_wait_ld_regs(r);
 #pragma unroll
-      for (int kk = 0; kk < kAttChunk / 16; ++kk)
-        tc_mma_bf16(tO, da + 2ull * kk, db + 2ull * kk, make_idesc_bf16(kAttHeads, kAttHalf),
-                    (kc > 0 || kk > 0) ? 1u : 0u);
-      tc_commit(&sm.pv_done[st]);
+        for (int j = 0; j < 32; j += 4)
+          *reinterpret_cast<float4*>(dst + cc * 32 + j) =
+              make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
+                          __uint_as_float(r[j + 3]));
+      }
+      if (v == 0) {
+        float* ml = p.ml + (static_cast<size_t>(b) * n_split + c) * 2 * kAttHeads;
+        ml[h] = sm.m[h];
+        ml[kAttHeads + h] = sm.l[h];
+      }
+      tc_fence_before();
     }
-    ++pv_issued[st];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) xa[i] = xb[i];
-  }
-  const int last_pv = (kAttPvChunks - 1) & 1;
-  if (ok) ok = mbar_wait(&sm.pv_done[last_pv], (pv_issued[last_pv] - 1) & 1u, ctl, DETAIL_WAIT_ACCFULL);
-  ok = !__syncthreads_or(!ok);
-
-  // 4. Unnormalised O, m and l of the split.
-  if (ok && warp < 4) {
-    tc_fence_after();
-    const uint32_t h = warp * 32u + lane;
-    const uint32_t lane_base = (warp * 32u) << 16;
-    float* dst = p.o_part + ((static_cast<size_t>(b) * n_split + c) * kAttHeads + h) * kAttDv + v * kAttHalf;
-    for (int cc = 0; cc < kAttHalf / 32; ++cc) {
-      uint32_t r[32];
-      tmem_ld_32x32b_x32(tO + lane_base + cc * 32, r);
-      tmem_wait_ld_regs(r);
-#pragma unroll
-      for (int j = 0; j < 32; j += 4)
-        *reinterpret_cast<float4*>(dst + cc * 32 + j) =
-            make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
-                        __uint_as_float(r[j + 3]));
-    }
-    if (v == 0) {
-      float* ml = p.ml + (static_cast<size_t>(b) * n_split + c) * 2 * kAttHeads;
-      ml[h] = sm.m[h];
-      ml[kAttHeads + h] = sm.l[h];
-    }
-    tc_fence_before();
+    __syncthreads();  // O is read before the next half's MMAs overwrite it
   }
   if (!ok && tid == 0) {
     // Let the MMAs this CTA issued land before its TMEM is freed (bounded).
@@ -392,7 +395,7 @@ dsa_status launch_attention(const AttentionLaunch& a) {
   if (cudaFuncSetAttribute(attention_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return DSA_ERR_CUDA;
-  attention_split_kernel<<<dim3(n_split, kAttDv / kAttHalf, a.B), kAttThreads, smem, a.stream>>>(p);
+  attention_split_kernel<<<dim3(n_split, 1, a.B), kAttThreads, smem, a.stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
   attention_combine_kernel<<<dim3(kAttHeads, a.B), 128, 0, a.stream>>>(p.o_part, p.ml, n_split,
                                                                         p.scale_log2, a.out);
