@@ -8,20 +8,22 @@
 //     out[b, h] = sum_s softmax_s(scale * q[b, h] . K[s]) V[s]  over the selected positions s.
 //
 // attention_split_kernel: CTA (c, b) takes the 256 selected positions c*256 .. c*256+255 of
-// request b. All operands are K-major bf16 tiles
-// in shared memory with the 128-byte swizzle, written by the CTA's threads (cp.async for the
-// query and key rows, register transposes for the values), and every product runs on the
-// tensor cores (tcgen05.mma kind::f16, FP32 accumulators in TMEM):
+// request b. All operands are bf16 tiles in shared memory with the 128-byte swizzle, written by
+// cp.async (zero-filled for unselected keys), and every product runs on the tensor cores
+// (tcgen05.mma kind::f16, FP32 accumulators in TMEM):
 //   1. S[128 heads][256 keys] = Q . K^T over the 576 dims, nine 64-dim chunks in three stages,
 //      loaded two chunks ahead (each chunk: four M=128, N=256, K=16 MMAs into TMEM columns
 //      0..255);
-//   2. four warps (thread = head) read S, mask unselected keys, and form the split's softmax
-//      numerators P = exp(scale (S - m)) in bf16 (shared memory, K-major) with the row max m
-//      and sum l in fp32;
-//   3. for each value half (dims 0..255, then 256..511): O[128][256] = P . V over the 256 keys,
-//      four 64-key chunks whose V^T tiles are built by transposing 8x8 blocks in registers
-//      (MMAs into TMEM columns 256..511, which S no longer needs), and the half of O goes to the
-//      workspace; m and l go with the first half.
+//   2. the loads of the first four value chunks start, then all eight warps read S (warp w:
+//      heads 32(w%4).., keys 128(w/4)..), mask unselected keys and form the split's softmax
+//      numerators P = exp(scale (S - m)) in bf16 (shared memory, K-major), with the row max m
+//      and the two partial sums of l exchanged through shared memory;
+//   3. O[128][512] = P . V over eight 32-key chunks: each chunk holds its keys' 512 value dims
+//      as they sit in the latent row (dims contiguous, the MN-major operand layout, no
+//      transposes), four slots of 32 KB loaded up to three chunks ahead; dims 0..255 accumulate
+//      in TMEM columns 256..511 and dims 256..511 in columns 0..255, which S no longer needs;
+//   4. warps 0..3 write O's first half, warps 4..7 its second, unnormalised, with m and l, to
+//      the workspace.
 // attention_combine_kernel then merges the splits of a request (log-sum-exp weights) into out.
 // Waits on the tensor core are bounded; a timeout is recorded as DSA_ERR_TIMEOUT.
 #include <algorithm>
@@ -37,32 +39,50 @@ namespace dsa {
 constexpr int kAttHeads = 128;
 constexpr int kAttDqk = 576;
 constexpr int kAttDv = 512;
-constexpr int kAttHalf = 256;             // value dims per CTA
+constexpr int kAttHalf = 256;             // value dims per accumulator (N of one MMA)
 constexpr int kAttSplit = 256;            // selected keys per CTA
-constexpr int kAttChunk = 64;             // dims per QK chunk, keys per PV chunk (128-byte rows)
+constexpr int kAttChunk = 64;             // dims per QK chunk (128-byte rows)
 constexpr int kAttThreads = 256;
 constexpr int kAttQkChunks = kAttDqk / kAttChunk;   // 9
-constexpr int kAttPvChunks = kAttSplit / kAttChunk;  // 4
-
 constexpr int kAttQkStages = 3;
+constexpr int kAttPvKeys = 32;                       // keys per value chunk
+constexpr int kAttPvChunks = kAttSplit / kAttPvKeys;  // 8
+constexpr int kAttPvSlots = 4;
+constexpr int kAttPvSlotBytes = kAttPvKeys * kAttDv * 2;  // 32 KB
+constexpr int kAttPvBlockBytes = kAttPvKeys * 128;         // one 64-dim column block of a chunk
 
 struct AttSmem {
-  // QK stages: Q chunk [128][64] + K chunk [256][64] bf16 each (48 KB); the two V^T stages
-  // [256 dims][64 keys] (32 KB each) reuse them once S is complete.
+  // QK stages: Q chunk [128][64] + K chunk [256][64] bf16 each (48 KB); once S is complete the
+  // first 128 KB hold the four value slots, each [8 column blocks of 64 dims][32 keys][64 dims].
   uint8_t stage[kAttQkStages][48 * 1024];
-  uint8_t p[kAttPvChunks][kAttHeads * 128];  // P [128 heads][256 keys] as four K-major 64-key chunks
-  int32_t rows[kAttSplit];                   // latent row of each selected key, -1: masked
-  float m[kAttHeads], l[kAttHeads];
-  uint64_t qk_done[kAttQkStages], pv_done[2];
+  uint8_t p[kAttSplit / 64][kAttHeads * 128];  // P [128 heads][256 keys] as four K-major 64-key chunks
+  int32_t rows[kAttSplit];                     // latent row of each selected key, -1: masked
+  float pm[2][kAttHeads], pl[2][kAttHeads];    // per key half: row max, sum of the rounded weights
+  uint64_t qk_done[kAttQkStages], pv_done[kAttPvSlots];
   uint32_t tmem;
   int abort;
 };
+static_assert(kAttPvSlots * kAttPvSlotBytes <= kAttQkStages * 48 * 1024, "value slots exceed the stages");
 
 __host__ __device__ constexpr uint32_t make_idesc_bf16(uint32_t M, uint32_t N) {
   return (1u << 4)                 // D format F32
          | (1u << 7) | (1u << 10)  // A, B format BF16
          | ((N >> 3) << 17)        // N / 8
          | ((M >> 4) << 24);       // M / 16
+}
+constexpr uint32_t kIdescBMnMajor = 1u << 16;  // B operand MN-major (N contiguous)
+
+// Shared-memory descriptor of an MN-major operand with the 128-byte swizzle: rows of 64
+// contiguous MN elements (128 bytes), eight K rows per 1024-byte atom; sbo = bytes between
+// groups of eight K rows, lbo = bytes between 64-element MN column blocks.
+__device__ __forceinline__ uint64_t make_smem_desc_mn(uint32_t smem_addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t desc = 0;
+  desc |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+  desc |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  desc |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  desc |= 1ull << 46;  // descriptor version
+  desc |= 2ull << 61;  // 128-byte swizzle
+  return desc;
 }
 
 __device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
@@ -99,7 +119,7 @@ struct AttParams {
   const int32_t* idx;         // [B][topk]
   int32_t n_blocks, block_size, max_blocks, B, topk;
   float scale_log2;           // scale * log2(e)
-  float* o_part;              // [B][n_split][128][512]
+  float* o_part;              // [B][n_split][512 dims][128 heads]
   float* ml;                  // [B][n_split][2][128]
   WsHeader* hdr;
   uint64_t budget_ns;
@@ -114,7 +134,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attention_split_kernel(const _
   const int n_split = gridDim.x;
   if (tid == 0) {
     for (int i = 0; i < kAttQkStages; ++i) mbar_init(&sm.qk_done[i], 1);
-    for (int i = 0; i < 2; ++i) mbar_init(&sm.pv_done[i], 1);
+    for (int i = 0; i < kAttPvSlots; ++i) mbar_init(&sm.pv_done[i], 1);
     fence_mbar_init();
     sm.abort = 0;
   }
@@ -148,7 +168,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attention_split_kernel(const _
   const WaitCtl ctl{p.hdr, &sm.abort, p.budget_ns};
   const uint16_t* qb = p.q + static_cast<size_t>(b) * kAttHeads * kAttDqk;
   bool ok = true;
-  uint32_t qk_issued[kAttQkStages] = {0, 0, 0}, pv_issued[2] = {0, 0};
+  uint32_t qk_issued[kAttQkStages] = {0, 0, 0}, pv_issued[kAttPvSlots] = {0, 0, 0, 0};
 
   // 1. S = Q K^T over nine 64-dim chunks, loads two chunks ahead of the MMAs (three stages).
   auto load_qk = [&](int ch) {
@@ -200,136 +220,148 @@ __global__ void __launch_bounds__(kAttThreads, 1) attention_split_kernel(const _
     ++qk_issued[st];
   }
   cp_async_wait<0>();  // nothing of this CTA's is still landing (also on the abort path)
-  // S complete: the last chunk's commit covers every earlier MMA.
+  // S complete: the last chunk's commit covers every earlier MMA, so the stages are free.
   const int last_qk = (kAttQkChunks - 1) % kAttQkStages;
   if (ok) ok = mbar_wait(&sm.qk_done[last_qk], (qk_issued[last_qk] - 1) & 1u, ctl, DETAIL_WAIT_ACCFULL);
   ok = !__syncthreads_or(!ok);
 
-  // 2. Softmax numerators of the split (warps 0..3, thread = head).
-  if (ok && warp < 4) {
+  // Value chunk i: keys i*32 .. i*32+31, all 512 value dims, into slot i % 4 as eight 64-dim
+  // column blocks of [32 keys][128 bytes]; a warp copies 512 contiguous bytes of one key.
+  auto load_v = [&](int i) {
+    uint8_t* slot = sm.stage[0] + (i % kAttPvSlots) * kAttPvSlotBytes;
+#pragma unroll
+    for (int it = 0; it < kAttPvSlotBytes / 16 / kAttThreads; ++it) {  // 8
+      const uint32_t u = tid + it * kAttThreads, r = u >> 6, j = u & 63u;
+      const int row = sm.rows[i * kAttPvKeys + r];
+      const uint16_t* src = p.latent + static_cast<size_t>(row < 0 ? 0 : row) * kAttDqk + j * 8;
+      cp_async_16(slot + (j >> 3) * kAttPvBlockBytes + sw128(r, j & 7u), src, row < 0 ? 0u : 16u);
+    }
+    cp_async_commit();
+  };
+  if (ok) {
+#pragma unroll
+    for (int i = 0; i < kAttPvSlots; ++i) load_v(i);
+  }
+
+  // 2. Softmax numerators of the split: warp w takes heads 32(w%4).. over keys 128(w/4)..
+  const uint32_t h = (warp & 3u) * 32u + lane, kh = warp >> 2;
+  const uint32_t lane_base = ((warp & 3u) * 32u) << 16;
+  if (ok) {
     tc_fence_after();
-    const uint32_t h = warp * 32u + lane;
-    const uint32_t lane_base = (warp * 32u) << 16;
     float mx = -INFINITY;
-    for (int cc = 0; cc < kAttSplit / 32; ++cc) {
+#pragma unroll 1
+    for (int cc = 0; cc < 4; ++cc) {
+      const int key0 = kh * 128 + cc * 32;
       uint32_t r[32];
-      tmem_ld_32x32b_x32(tS + lane_base + cc * 32, r);
+      tmem_ld_32x32b_x32(tS + lane_base + key0, r);
       tmem_wait_ld_regs(r);
 #pragma unroll
       for (int j = 0; j < 32; ++j)
-        if (sm.rows[cc * 32 + j] >= 0) mx = fmaxf(mx, __uint_as_float(r[j]));
+        if (sm.rows[key0 + j] >= 0) mx = fmaxf(mx, __uint_as_float(r[j]));
     }
+    sm.pm[kh][h] = mx;
+    __syncthreads();
+    mx = fmaxf(sm.pm[0][h], sm.pm[1][h]);
     float sum = 0.0f;
-    for (int cc = 0; cc < kAttSplit / 32; ++cc) {
+#pragma unroll 1
+    for (int cc = 0; cc < 4; ++cc) {
+      const int key0 = kh * 128 + cc * 32;
       uint32_t r[32];
-      tmem_ld_32x32b_x32(tS + lane_base + cc * 32, r);
+      tmem_ld_32x32b_x32(tS + lane_base + key0, r);
       tmem_wait_ld_regs(r);
       uint32_t packed[16];
 #pragma unroll
       for (int j = 0; j < 32; j += 2) {
-        const bool v0 = sm.rows[cc * 32 + j] >= 0, v1 = sm.rows[cc * 32 + j + 1] >= 0;
+        const bool v0 = sm.rows[key0 + j] >= 0, v1 = sm.rows[key0 + j + 1] >= 0;
         const float p0 = v0 ? exp2f((__uint_as_float(r[j]) - mx) * p.scale_log2) : 0.0f;
         const float p1 = v1 ? exp2f((__uint_as_float(r[j + 1]) - mx) * p.scale_log2) : 0.0f;
         const __nv_bfloat162 pp = __floats2bfloat162_rn(p0, p1);
         sum += __low2float(pp) + __high2float(pp);  // the weights the value product uses
         packed[j >> 1] = *reinterpret_cast<const uint32_t*>(&pp);
       }
-      // keys cc*32 .. cc*32+31: chunk cc/2, units (cc&1)*4 .. +3 of row h
-      uint8_t* pc = sm.p[cc >> 1];
+      // keys key0 .. key0+31: P chunk key0/64, units (key0/32 & 1)*4 .. +3 of row h
+      uint8_t* pc = sm.p[key0 >> 6];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const uint4 w4 = make_uint4(packed[4 * u], packed[4 * u + 1], packed[4 * u + 2], packed[4 * u + 3]);
-        *reinterpret_cast<uint4*>(pc + sw128(h, (cc & 1) * 4 + u)) = w4;
+        *reinterpret_cast<uint4*>(pc + sw128(h, ((key0 >> 5) & 1) * 4 + u)) = w4;
       }
     }
-    sm.m[h] = mx;
-    sm.l[h] = sum;
+    sm.pl[kh][h] = sum;
     tc_fence_before();
   }
   fence_proxy_async_smem();
-  __syncthreads();
 
-  // 3. and 4., once per value half v: O = P V over four 64-key chunks into TMEM columns
-  // 256..511 (V^T chunks built by 8x8 register transposes, the next chunk's rows loading while
-  // the current one is transposed), then the unnormalised O of the half to the workspace.
-  const uint32_t ko = tid & 7u, dO = tid >> 3;  // key octet, dim octet (32 of them: 256 dims)
-  auto load_v = [&](int v, int kc, uint4 (&x)[8]) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int row = sm.rows[kc * kAttChunk + ko * 8 + i];
-      x[i] = row < 0 ? make_uint4(0u, 0u, 0u, 0u)
-                     : __ldg(reinterpret_cast<const uint4*>(p.latent + static_cast<size_t>(row) * kAttDqk +
-                                                            v * kAttHalf + dO * 8));
-    }
-  };
-  uint4 xa[8], xb[8];
-  for (int v = 0; v < kAttDv / kAttHalf && ok; ++v) {
-    load_v(v, 0, xa);
-    for (int kc = 0; kc < kAttPvChunks && ok; ++kc) {
-      const int st = kc & 1;
-      if (pv_issued[st] > 0) ok = mbar_wait(&sm.pv_done[st], (pv_issued[st] - 1) & 1u, ctl, DETAIL_WAIT_ACCFULL);
-      if (__syncthreads_or(!ok)) { ok = false; break; }
-      if (kc + 1 < kAttPvChunks) load_v(v, kc + 1, xb);
-      uint8_t* vt = sm.stage[st];  // [256 dims][64 keys]
-      // xa[i] holds dims dO*8 .. +7 of key i; row e of the block gathers dim e of keys 0..7.
-      const uint32_t* xw = reinterpret_cast<const uint32_t*>(xa);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        uint32_t w[4];
-#pragma unroll
-        for (int k2 = 0; k2 < 4; ++k2) {
-          const uint32_t a = xw[(2 * k2) * 4 + (e >> 1)], bb = xw[(2 * k2 + 1) * 4 + (e >> 1)];
-          w[k2] = __byte_perm(a, bb, (e & 1) ? 0x7632u : 0x5410u);
-        }
-        *reinterpret_cast<uint4*>(vt + sw128(dO * 8 + e, ko)) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-      fence_proxy_async_smem();
-      __syncthreads();
-      if (tid == 0) {
-        tc_fence_after();
-        const uint64_t da = make_smem_desc(smem_u32(sm.p[kc]), 128), db = make_smem_desc(smem_u32(vt), 128);
-#pragma unroll
-        for (int kk = 0; kk < kAttChunk / 16; ++kk)
-          tc_mma_bf16(tO, da + 2ull * kk, db + 2ull * kk, make_idesc_bf16(kAttHeads, kAttHalf),
-                      (kc > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(&sm.pv_done[st]);
-      }
-      ++pv_issued[st];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) xa[i] = xb[i];
-    }
-    const int last_pv = (kAttPvChunks - 1) & 1;
-    if (ok) ok = mbar_wait(&sm.pv_done[last_pv], (pv_issued[last_pv] - 1) & 1u, ctl, DETAIL_WAIT_ACCFULL);
-    ok = !__syncthreads_or(!ok);
-    if (ok && warp < 4) {
+  // 3. O = P V over eight 32-key chunks; dims 0..255 into columns 256..511, dims 256..511 into
+  // columns 0..255. After issuing chunk i (1 <= i <= 4), slot (i-1) % 4 is refilled with chunk
+  // i+3 once the MMAs of chunk i-1 have read it.
+  const uint32_t idesc_pv = make_idesc_bf16(kAttHeads, kAttHalf) | kIdescBMnMajor;
+#pragma unroll 1
+  for (int i = 0; i < kAttPvChunks && ok; ++i) {
+    // this thread's copies of chunk i have landed; the newer groups may still be in flight
+    if (i == 0) cp_async_wait<3>();
+    else if (i <= 5) cp_async_wait<2>();
+    else if (i == 6) cp_async_wait<1>();
+    else cp_async_wait<0>();
+    fence_proxy_async_smem();
+    if (__syncthreads_or(!ok)) { ok = false; break; }
+    const int slot = i % kAttPvSlots;
+    if (tid == 0) {
       tc_fence_after();
-      const uint32_t h = warp * 32u + lane;
-      const uint32_t lane_base = (warp * 32u) << 16;
-      float* dst = p.o_part + ((static_cast<size_t>(b) * n_split + c) * kAttHeads + h) * kAttDv + v * kAttHalf;
-      for (int cc = 0; cc < kAttHalf / 32; ++cc) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tO + lane_base + cc * 32, r);
-        tmem_wait_ld_regs(r);
+      const uint32_t vbase = smem_u32(sm.stage[0] + slot * kAttPvSlotBytes);
+      const uint64_t da = make_smem_desc(smem_u32(sm.p[i >> 1]), 128);
 #pragma unroll
-        for (int j = 0; j < 32; j += 4)
-          *reinterpret_cast<float4*>(dst + cc * 32 + j) =
-              make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
-                          __uint_as_float(r[j + 3]));
+      for (int half = 0; half < kAttDv / kAttHalf; ++half) {
+#pragma unroll
+        for (int kk = 0; kk < kAttPvKeys / 16; ++kk) {
+          const uint64_t db = make_smem_desc_mn(vbase + half * 4 * kAttPvBlockBytes + kk * 2048,
+                                                kAttPvBlockBytes, 1024);
+          tc_mma_bf16(half == 0 ? tO : tS, da + 2ull * ((i & 1) * 2 + kk), db, idesc_pv,
+                      (i > 0 || kk > 0) ? 1u : 0u);
+        }
       }
-      if (v == 0) {
-        float* ml = p.ml + (static_cast<size_t>(b) * n_split + c) * 2 * kAttHeads;
-        ml[h] = sm.m[h];
-        ml[kAttHeads + h] = sm.l[h];
-      }
-      tc_fence_before();
+      tc_commit(&sm.pv_done[slot]);
     }
-    __syncthreads();  // O is read before the next half's MMAs overwrite it
+    ++pv_issued[slot];
+    if (i >= 1 && i + 3 < kAttPvChunks) {
+      const int sp = (i - 1) % kAttPvSlots;
+      ok = mbar_wait(&sm.pv_done[sp], (pv_issued[sp] - 1) & 1u, ctl, DETAIL_WAIT_ACCFULL);
+      if (__syncthreads_or(!ok)) { ok = false; break; }
+      load_v(i + 3);
+    }
+  }
+  cp_async_wait<0>();
+  const int last_pv = (kAttPvChunks - 1) % kAttPvSlots;
+  if (ok) ok = mbar_wait(&sm.pv_done[last_pv], (pv_issued[last_pv] - 1) & 1u, ctl, DETAIL_WAIT_ACCFULL);
+  ok = !__syncthreads_or(!ok);
+
+  // 4. The unnormalised O of the split with m and l: warps 0..3 dims 0..255 (columns
+  // 256..511), warps 4..7 dims 256..511 (columns 0..255). The partials are stored dim-major
+  // ([dim][head]), so each store of a warp writes 128 contiguous bytes.
+  if (ok) {
+    tc_fence_after();
+    float* dst = p.o_part + ((static_cast<size_t>(b) * n_split + c) * kAttDv + kh * kAttHalf) * kAttHeads + h;
+    const uint32_t tcol = kh == 0 ? tO : tS;
+#pragma unroll 1
+    for (int cc = 0; cc < kAttHalf / 32; ++cc) {
+      uint32_t r[32];
+      tmem_ld_32x32b_x32(tcol + lane_base + cc * 32, r);
+      tmem_wait_ld_regs(r);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) dst[(cc * 32 + j) * kAttHeads] = __uint_as_float(r[j]);
+    }
+    if (kh == 0) {
+      float* ml = p.ml + (static_cast<size_t>(b) * n_split + c) * 2 * kAttHeads;
+      ml[h] = fmaxf(sm.pm[0][h], sm.pm[1][h]);
+      ml[kAttHeads + h] = sm.pl[0][h] + sm.pl[1][h];
+    }
+    tc_fence_before();
   }
   if (!ok && tid == 0) {
     // Let the MMAs this CTA issued land before its TMEM is freed (bounded).
     for (int i = 0; i < kAttQkStages; ++i)
       if (qk_issued[i]) mbar_wait_drain(&sm.qk_done[i], (qk_issued[i] - 1) & 1u, p.budget_ns);
-    for (int i = 0; i < 2; ++i)
+    for (int i = 0; i < kAttPvSlots; ++i)
       if (pv_issued[i]) mbar_wait_drain(&sm.pv_done[i], (pv_issued[i] - 1) & 1u, p.budget_ns);
   }
   __syncthreads();
@@ -340,29 +372,76 @@ __global__ void __launch_bounds__(kAttThreads, 1) attention_split_kernel(const _
 }
 
 // out[b][h][d] = sum_c e^(m_c - M) O_c[h][d] / sum_c e^(m_c - M) l_c over the request's splits
-// (M the largest m_c); a head whose splits selected nothing gets zeros.
-__global__ void __launch_bounds__(128) attention_combine_kernel(const float* __restrict__ o_part,
-                                                                const float* __restrict__ ml, int n_split,
+// (M the largest m_c); a head whose splits selected nothing gets zeros. Block (x, b) takes dims
+// 16x .. 16x+15 of all 128 heads: the partials are read along heads, 16 bytes a thread with
+// every split's loads in flight at once, and out is written in 64-byte runs.
+constexpr int kCombineDims = 16;
+constexpr int kMaxSplits = DSA_MAX_TOPK / kAttSplit;
+template <int NS>
+__global__ void __launch_bounds__(256) attention_combine_kernel(const float* __restrict__ o_part,
+                                                                const float* __restrict__ ml,
                                                                 float scale_log2, float* __restrict__ out) {
-  const int h = blockIdx.x, b = blockIdx.y;
-  float M = -INFINITY;
-  for (int c = 0; c < n_split; ++c)
-    M = fmaxf(M, ml[(static_cast<size_t>(b) * n_split + c) * 2 * kAttHeads + h]);
-  float wsum = 0.0f;
-  float w[DSA_MAX_TOPK / kAttSplit];
-  for (int c = 0; c < n_split; ++c) {
-    const float* mlc = ml + (static_cast<size_t>(b) * n_split + c) * 2 * kAttHeads;
-    const float mc = mlc[h];
-    w[c] = (mc == -INFINITY) ? 0.0f : exp2f((mc - M) * scale_log2);
-    wsum += w[c] * mlc[kAttHeads + h];
+  constexpr int n_split = NS;
+  __shared__ __align__(16) float wt[NS][kAttHeads];
+  __shared__ float tile[kCombineDims][kAttHeads + 1];
+  const int d0 = blockIdx.x * kCombineDims, b = blockIdx.y;
+  const int tid = threadIdx.x;
+  static_assert(NS >= 1 && NS <= kMaxSplits, "splits per request");
+  const float* mlb = ml + static_cast<size_t>(b) * n_split * 2 * kAttHeads;
+  if (tid < kAttHeads) {
+    const int h = tid;
+    float mc[NS], lc[NS];
+#pragma unroll
+    for (int c = 0; c < NS; ++c) {
+      mc[c] = mlb[c * 2 * kAttHeads + h];
+      lc[c] = mlb[c * 2 * kAttHeads + kAttHeads + h];
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < NS; ++c) M = fmaxf(M, mc[c]);
+    float wsum = 0.0f;
+#pragma unroll
+    for (int c = 0; c < NS; ++c) {
+      mc[c] = (mc[c] == -INFINITY) ? 0.0f : exp2f((mc[c] - M) * scale_log2);
+      wsum += mc[c] * lc[c];
+    }
+    const float inv = wsum > 0.0f ? 1.0f / wsum : 0.0f;
+#pragma unroll
+    for (int c = 0; c < NS; ++c) wt[c][h] = mc[c] * inv;
   }
-  const float inv = wsum > 0.0f ? 1.0f / wsum : 0.0f;
-  for (int d = threadIdx.x; d < kAttDv; d += 128) {
-    float acc = 0.0f;
-    for (int c = 0; c < n_split; ++c)
-      acc += w[c] * o_part[((static_cast<size_t>(b) * n_split + c) * kAttHeads + h) * kAttDv + d];
-    out[(static_cast<size_t>(b) * kAttHeads + h) * kAttDv + d] = acc * inv;
+  __syncthreads();
+  {
+    // thread: heads 4(t%32) .. +3, dims d0 + 2(t/32), +1; a warp reads 512 contiguous bytes
+    const int hq = tid & 31, dd = tid >> 5;
+    const float* src = o_part + (static_cast<size_t>(b) * n_split * kAttDv + d0 + 2 * dd) * kAttHeads + 4 * hq;
+    float4 v[NS][2];
+#pragma unroll
+    for (int c = 0; c < NS; ++c)
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+        v[c][j] = __ldcs(reinterpret_cast<const float4*>(src + (static_cast<size_t>(c) * kAttDv + j) * kAttHeads));
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+      for (int c = 0; c < NS; ++c) {
+        const float4 w = *reinterpret_cast<const float4*>(&wt[c][4 * hq]);
+        acc.x += w.x * v[c][j].x;
+        acc.y += w.y * v[c][j].y;
+        acc.z += w.z * v[c][j].z;
+        acc.w += w.w * v[c][j].w;
+      }
+      float* trow = tile[2 * dd + j] + 4 * hq;
+      trow[0] = acc.x;
+      trow[1] = acc.y;
+      trow[2] = acc.z;
+      trow[3] = acc.w;
+    }
   }
+  __syncthreads();
+  const int lane = tid & 31, warp = tid >> 5;
+  for (int h = warp * 2 + (lane >> 4); h < kAttHeads; h += 16)
+    out[(static_cast<size_t>(b) * kAttHeads + h) * kAttDv + d0 + (lane & 15)] = tile[lane & 15][h];
 }
 
 size_t attention_workspace_bytes(int B, int topk) {
@@ -374,6 +453,7 @@ size_t attention_workspace_bytes(int B, int topk) {
 
 dsa_status launch_attention(const AttentionLaunch& a) {
   const int n_split = a.topk / kAttSplit;
+  if (n_split < 1 || n_split > kMaxSplits || a.topk % kAttSplit != 0) return DSA_ERR_UNSUPPORTED;
   uint8_t* base = static_cast<uint8_t*>(a.ws);
   AttParams p;
   p.q = a.q;
@@ -397,8 +477,17 @@ dsa_status launch_attention(const AttentionLaunch& a) {
     return DSA_ERR_CUDA;
   attention_split_kernel<<<dim3(n_split, 1, a.B), kAttThreads, smem, a.stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
-  attention_combine_kernel<<<dim3(kAttHeads, a.B), 128, 0, a.stream>>>(p.o_part, p.ml, n_split,
-                                                                        p.scale_log2, a.out);
+  const dim3 cgrid(kAttDv / kCombineDims, a.B);
+  switch (n_split) {
+#define DSA_COMBINE_CASE(NS)                                                                   \
+  case NS:                                                                                     \
+    attention_combine_kernel<NS><<<cgrid, 256, 0, a.stream>>>(p.o_part, p.ml, p.scale_log2, a.out); \
+    break;
+    DSA_COMBINE_CASE(1) DSA_COMBINE_CASE(2) DSA_COMBINE_CASE(3) DSA_COMBINE_CASE(4)
+    DSA_COMBINE_CASE(5) DSA_COMBINE_CASE(6) DSA_COMBINE_CASE(7) DSA_COMBINE_CASE(8)
+#undef DSA_COMBINE_CASE
+    default: return DSA_ERR_UNSUPPORTED;
+  }
   return cuda_status(cudaGetLastError());
 }
 

@@ -36,7 +36,7 @@ def _check(x, got, scale):
 
 
 @pytest.mark.parametrize("lens,topk", [([3000, 700, 256, 40], 256), ([5000, 2048, 1, 9000], 512),
-                                       ([30000, 4000], 2048)])
+                                       ([4000, 900, 12000], 768), ([30000, 4000], 2048)])
 def test_matches_oracle(lens, topk):
     x = latent_decode_inputs(lens, topk, seed=sum(lens) % 1000)
     scale = 1.0 / np.sqrt(576.0)
