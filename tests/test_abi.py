@@ -96,3 +96,37 @@ def test_decode_workspace_size_matches_its_documented_layout(lib):
         assert binding.dsa_decode_workspace_bytes(B, max_len, 64, 128, 2048) == want, (B, max_len)
     n_req, n_scores = binding.DSA_NOALLOC_MAX_REQUESTS, binding.DSA_NOALLOC_MAX_SCORES
     assert binding.dsa_decode_workspace_bytes(n_req, n_scores // n_req, 64, 128, 2048) == 34 * 2**20 + 4352
+
+
+def test_sparse_attention_workspace_and_host_validation(lib):
+    """The attention workspace is the header, then [B][topk/256][512][128] fp32 partials and
+    [B][topk/256][2][128] fp32 row maxima and sums; unsupported shapes and malformed arguments
+    are rejected on the host, before anything is enqueued."""
+    for B, topk in ((1, 256), (3, 768), (32, 2048)):
+        n_split = topk // 256
+        want = binding.DSA_WS_HEADER_BYTES + B * n_split * 512 * 128 * 4 + B * n_split * 2 * 128 * 4
+        assert lib.dsa_sparse_attention_workspace_bytes(B, topk) == want
+    for B, topk in ((0, 256), (1, 0), (1, 300), (1, 2304)):
+        assert lib.dsa_sparse_attention_workspace_bytes(B, topk) == 0
+
+    p = ctypes.c_void_p(1 << 20)  # never dereferenced: every case below returns first
+    f = lib.dsa_sparse_attention_decode
+
+    def call(q=p, latent=p, n_blocks=4, block_size=64, table=p, max_blocks=4, seq=p, idx=p, B=2,
+             Hq=128, dqk=576, dv=512, topk=256, scale=0.05, out=p, ws=None, ws_bytes=0):
+        return f(q, latent, n_blocks, block_size, table, max_blocks, seq, idx, B, Hq, dqk, dv, topk,
+                 scale, out, ws, ws_bytes, None)
+
+    assert call(q=None) == binding.DSA_ERR_INVALID
+    assert call(idx=None) == binding.DSA_ERR_INVALID
+    assert call(B=0) == binding.DSA_ERR_INVALID
+    assert call(scale=0.0) == binding.DSA_ERR_INVALID
+    assert call(scale=float("nan")) == binding.DSA_ERR_INVALID
+    assert call(q=ctypes.c_void_p((1 << 20) + 8)) == binding.DSA_ERR_INVALID   # not 16-byte aligned
+    assert call(Hq=64) == binding.DSA_ERR_UNSUPPORTED
+    assert call(dqk=512) == binding.DSA_ERR_UNSUPPORTED
+    assert call(topk=300) == binding.DSA_ERR_UNSUPPORTED
+    assert call(topk=4096) == binding.DSA_ERR_UNSUPPORTED
+    assert call() == binding.DSA_ERR_INVALID                                   # no workspace
+    need = lib.dsa_sparse_attention_workspace_bytes(2, 256)
+    assert call(ws=p, ws_bytes=need - 1) == binding.DSA_ERR_INVALID            # too small
