@@ -714,6 +714,7 @@ def cpu_baseline_long(lp, seconds):
         res[name] = (pairs, n, time.perf_counter() - t0)
     p1, n1, e1 = res["single"]
     pa, na, ea = res["all"]
+    step_pairs = 12 * causal_pairs(lp.L)
     return {"value": p1 / e1, "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"{n1} uniformly drawn query rows of indexer layer 0 of the 200000-token "
                       f"workload ({p1} causal pairs, {e1:.1f} s) through the plain single-threaded "
@@ -721,7 +722,20 @@ def cpu_baseline_long(lp, seconds):
             "all_cores": {"value": pa / ea, "unit": UNIT, "cores": nproc,
                           "sample": f"{na} more rows ({pa} pairs, {ea:.1f} s), the same per-row "
                                     f"oracle on {nproc} threads over rows; checked the same way"},
-            "host_nproc": nproc}
+            "host_nproc": nproc,
+            "extrapolated_step_s": {
+                "single": extrapolated_seconds(step_pairs, p1, e1),
+                "all_cores": extrapolated_seconds(step_pairs, pa, ea),
+                "note": "one step of the headline workload (12 indexer layers x L(L+1)/2 causal pairs) "
+                        "at the sampled rates: extrapolated, not run (a row's cost grows with its "
+                        "position, and the rows are uniformly drawn)"}}
+
+
+def extrapolated_seconds(total_pairs, sampled_pairs, sampled_seconds):
+    """Seconds for total_pairs at the rate of a sample (None for an empty sample)."""
+    if sampled_pairs <= 0 or sampled_seconds <= 0:
+        return None
+    return total_pairs * sampled_seconds / sampled_pairs
 
 
 # ------------------------------------------------------------------------------------------

@@ -61,3 +61,13 @@ def test_reference_arm_runs_on_rank0_only():
                           "--gpus", "2", "--steps", "1", "--warmup", "3"],
                          capture_output=True, text=True, env=env, timeout=120)
     assert res.returncode == 0 and res.stdout.strip() == ""
+
+
+def test_cpu_baseline_extrapolation():
+    """The CPU baseline's full-step figure scales the sampled rate to the step's pairs."""
+    sys.path.insert(0, ROOT)
+    import bench
+    step = 12 * bench.causal_pairs(200000)
+    assert step == 12 * 200000 * 200001 // 2
+    assert bench.extrapolated_seconds(step, step // 4, 2.0) == pytest.approx(8.0, rel=1e-12)
+    assert bench.extrapolated_seconds(step, 0, 2.0) is None
