@@ -6,7 +6,6 @@ that source layer's plain indexer output, with every layer's indices kept and wi
 two buffers that the indexers keep rewriting. One source layer is also checked against the
 oracle."""
 
-import numpy as np
 import pytest
 import torch
 

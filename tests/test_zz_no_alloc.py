@@ -11,7 +11,6 @@ This file is collected last on purpose: it exercises the library's one fixed scr
 and must pass both alone in a fresh process and after every other test.
 """
 
-import numpy as np
 import pytest
 import torch
 
